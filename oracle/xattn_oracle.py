@@ -1,0 +1,286 @@
+"""CPU fp64 oracle for XAttention block-sparse prefill attention.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the package smoke check and the bench's
+CPU-baseline / reference legs may import or run this module. The product path
+(the CUDA library and its Python binding) never calls it and shares no code with
+it; the two meet only in the seeded input generators of `synthetic`.
+
+Everything here is plain, slow and meant to be checked by eye against the pages.
+Inputs arrive as bf16 bit patterns (uint16) and are widened exactly to fp64; all
+arithmetic is fp64. Library primitives used as single steps: numpy matmul, sort,
+exp/log.
+
+Passages followed (page title, section):
+- DuSA rebuttal (paperhub tM5mjMfFmS), "Response to Q2": Q and K of shape
+  (B, H, M, C) are reshaped to (B, H, M//stride, stride*C), and attention with a
+  softmax over the last two dimensions is computed on the reshaped tensors.
+- XAttention abstract (arXiv 2503.16428): the importance proxy is the sum of
+  antidiagonal values, running from the lower-left to the upper-right.
+- XAttention summary (atlas.scime.ai), "Approach": sum the strided antidiagonal
+  values inside each attention block; keep the minimal set of blocks whose
+  softmax-normalised antidiagonal mass exceeds a per-head threshold.
+- XAttention summary, "Measured effects" table: threshold selection versus Top-K
+  and fixed-ratio selection; strides 4, 8, 16, 64; diagonal vs antidiagonal.
+- FlexPrefill rebuttal (paperhub OfjIlbelrT), "R Q3" (Steps 6-7 of its Lagrangian
+  dual argument): the smallest index set whose normalised mass reaches the
+  cumulative threshold is the one taken greedily in descending score order.
+- DuSA rebuttal, "Response to W3"/"Response to Q1": attention is then performed
+  only within the important (kept) blocks.
+
+Readings where the pages are silent (each is exercised by the pins in tests/):
+- scoring scale sigma: an argument; default 1/sqrt(stride*C), the ordinary
+  attention scale of the reshaped head dimension stride*C.
+- causal scoring masks at the reshaped granularity: reshaped column j' is visible
+  to reshaped row i' iff j' <= i' (the i' = j' entry keeps its full antidiagonal).
+- block score = (1/g) * sum of the g x g softmax entries of a (query block,
+  key block) pair, g = block/stride, so each block row sums to 1.
+- "exceeds": the greedy prefix stops at the first block whose inclusion brings
+  the cumulative mass to >= tau; tau >= 1 keeps every candidate.
+- ties: descending score, then ascending block index.
+- the diagonal block is added after thresholding if it is not already kept.
+- GQA: query head h scores against KV head h // (Hq/Hkv), with its own tau_h.
+- sparse attention scale 1/sqrt(C); causal mask j <= i at token granularity.
+
+Parity pins for every function live in tests/test_oracle_pins.py; none of them
+re-types a formula from this file.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "bf16_to_f64", "default_score_scale", "strided_views", "antidiagonal_logits",
+    "block_scores", "select_row", "select_blocks", "selection_margins", "to_csr",
+    "block_sparse_attention", "dense_attention", "layer_block_scores",
+    "layer_select", "layer_sparse_attention",
+]
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bf16 bit patterns as fp64 (bf16 is the top half of fp32)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def default_score_scale(stride: int, C: int) -> float:
+    """1/sqrt(stride*C): the usual attention scale for the reshaped width stride*C."""
+    return 1.0 / np.sqrt(stride * C)
+
+
+# --------------------------------------------------------------------------- a1
+def strided_views(q: np.ndarray, k: np.ndarray, stride: int, antidiagonal: bool = True):
+    """Reshape q, k [M, C] to [M/stride, stride*C] (DuSA rebuttal, Response to Q2).
+
+    Row i' of the key view concatenates tokens i'*S, i'*S+1, ..., i'*S+S-1.
+    For antidiagonal scoring the query view concatenates the same S tokens in
+    reverse order (i'*S+S-1 first), so that chunk s of a query row meets chunk s
+    of a key row at token pair (i'*S+S-1-s, j'*S+s): the S x S tile's entries
+    from its lower-left corner to its upper-right corner (XAttention abstract).
+    With antidiagonal=False both views are forward, which gives the diagonal
+    pattern the DuSA rebuttal compares against.
+    """
+    M, C = q.shape
+    if M % stride:
+        raise ValueError("M must be a multiple of stride")
+    r = M // stride
+    q3 = q.reshape(r, stride, C)
+    if antidiagonal:
+        q3 = q3[:, ::-1, :]
+    qv = np.ascontiguousarray(q3).reshape(r, stride * C)
+    kv = np.ascontiguousarray(k.reshape(r, stride, C)).reshape(r, stride * C)
+    return qv, kv
+
+
+# --------------------------------------------------------------------------- a2
+def antidiagonal_logits(q, k, stride: int, sigma: float, causal: bool, antidiagonal: bool = True):
+    """X[i', j'] = sigma * <Q'[i'], K'[j']>, -inf where causal hides j' > i'.
+
+    Materialises the whole (M/S)^2 matrix: small inputs only.
+    """
+    qv, kv = strided_views(q, k, stride, antidiagonal)
+    X = sigma * (qv @ kv.T)
+    if causal:
+        r = X.shape[0]
+        X[np.triu_indices(r, 1)] = -np.inf
+    return X
+
+
+# ------------------------------------------------------------------------ a3+a4
+def block_scores(q, k, stride: int, block: int, sigma: float, causal: bool,
+                 rows=None, antidiagonal: bool = True, chunk_blocks: int = 8):
+    """Per-(query block, key block) softmax-normalised antidiagonal mass.
+
+    For every reshaped query row the softmax runs over all of its visible
+    reshaped key columns (the full row), then the g x g entries of each block
+    pair are summed and divided by g = block/stride, so that each block row sums
+    to 1. Returns an [nb, nb] fp64 array (rows not in `rows` are left NaN;
+    causal entries c > r are 0).
+    """
+    M, C = q.shape
+    if block % stride:
+        raise ValueError("block must be a multiple of stride")
+    nb, g = M // block, block // stride
+    qv, kv = strided_views(q, k, stride, antidiagonal)
+    out = np.full((nb, nb), np.nan)
+    rows = list(range(nb)) if rows is None else sorted(set(int(r) for r in rows))
+    for i in range(0, len(rows), chunk_blocks):
+        chunk = rows[i:i + chunk_blocks]
+        for r in chunk:
+            ri = slice(r * g, (r + 1) * g)
+            ncol = (r + 1) * g if causal else nb * g
+            X = sigma * (qv[ri] @ kv[:ncol].T)                 # [g, ncol]
+            if causal:
+                ii = np.arange(r * g, (r + 1) * g)[:, None]
+                jj = np.arange(ncol)[None, :]
+                X = np.where(jj <= ii, X, -np.inf)
+            X = X - X.max(axis=1, keepdims=True)               # row softmax (fp64)
+            P = np.exp(X)
+            P /= P.sum(axis=1, keepdims=True)
+            ncb = ncol // g
+            mass = P.reshape(g, ncb, g).sum(axis=(0, 2)) / g     # sum g x g, / g
+            out[r, :] = 0.0
+            out[r, :ncb] = mass
+    return out
+
+
+# --------------------------------------------------------------------------- a5
+def _candidates(r: int, nb: int, causal: bool) -> np.ndarray:
+    return np.arange(r + 1) if causal else np.arange(nb)
+
+
+def _greedy_order(row: np.ndarray, cand: np.ndarray) -> np.ndarray:
+    """Candidates in descending score, ties to the smaller block index."""
+    return cand[np.lexsort((cand, -row[cand]))]
+
+
+def select_row(row: np.ndarray, r: int, tau: float, causal: bool) -> np.ndarray:
+    """Kept key blocks of query block r, ascending.
+
+    Greedy prefix of the descending order, stopping at the first block whose
+    inclusion brings the cumulative mass to >= tau (the minimal set whose mass
+    reaches tau: FlexPrefill rebuttal R Q3; XAttention summary, Approach); tau >= 1
+    keeps every candidate; then the diagonal block r is added if missing.
+    """
+    nb = row.shape[0]
+    cand = _candidates(r, nb, causal)
+    if tau >= 1.0:
+        kept = list(cand)
+    else:
+        kept, cum = [], 0.0
+        for c in _greedy_order(row, cand):
+            kept.append(int(c))
+            cum += row[c]
+            if cum >= tau:
+                break
+    if r not in kept:
+        kept.append(r)
+    return np.array(sorted(kept), dtype=np.int64)
+
+
+def selection_margins(row: np.ndarray, r: int, tau: float, causal: bool):
+    """For each candidate block c: (cum_before(c) - tau, position in greedy order).
+
+    cum_before(c) is the mass of the blocks ahead of c in the descending order;
+    with tau < 1, c is kept by thresholding iff cum_before(c) < tau. Used to
+    classify GPU/oracle mask differences that rounding may legitimately flip.
+    """
+    nb = row.shape[0]
+    cand = _candidates(r, nb, causal)
+    order = _greedy_order(row, cand)
+    before = np.concatenate([[0.0], np.cumsum(row[order])[:-1]])
+    margin = np.full(nb, np.nan)
+    pos = np.full(nb, -1, dtype=np.int64)
+    margin[order] = before - tau
+    pos[order] = np.arange(order.size)
+    return margin, pos
+
+
+def select_blocks(scores: np.ndarray, tau: float, causal: bool, rows=None):
+    """select_row for each query block of one head; returns {r: kept}."""
+    nb = scores.shape[0]
+    rows = range(nb) if rows is None else rows
+    return {int(r): select_row(scores[r], int(r), tau, causal) for r in rows}
+
+
+def to_csr(kept_per_row):
+    """Concatenate per-row kept lists (in row order) into (row_ptr, col_idx) int32."""
+    counts = [len(k) for k in kept_per_row]
+    row_ptr = np.zeros(len(counts) + 1, np.int64)
+    row_ptr[1:] = np.cumsum(counts)
+    col = np.concatenate(kept_per_row) if kept_per_row else np.zeros(0)
+    return row_ptr.astype(np.int32), col.astype(np.int32)
+
+
+# --------------------------------------------------------------------------- a6
+def block_sparse_attention(q, k, v, kept, block: int, causal: bool, scale: float, rows=None):
+    """Softmax attention restricted to the kept key blocks of each query block.
+
+    kept: {r: ascending key-block indices}. Token i of query block r attends to
+    tokens j of its kept blocks (and j <= i when causal), with logits
+    scale * q_i . k_j; two-pass softmax in fp64. Returns (O [len(rows)*block, C],
+    lse [len(rows)*block]) in the order of `rows`; lse is natural-log.
+    """
+    M, C = q.shape
+    nb = M // block
+    rows = range(nb) if rows is None else rows
+    O, L = [], []
+    for r in rows:
+        cols = np.asarray(kept[int(r)], dtype=np.int64)
+        keys = (cols[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+        qi = q[r * block:(r + 1) * block]
+        logits = scale * (qi @ k[keys].T)
+        if causal:
+            ii = np.arange(r * block, (r + 1) * block)[:, None]
+            logits = np.where(keys[None, :] <= ii, logits, -np.inf)
+        m = logits.max(axis=1, keepdims=True)                  # pass 1: row max
+        p = np.exp(logits - m)                                 # pass 2: exp, sum
+        den = p.sum(axis=1, keepdims=True)
+        O.append((p @ v[keys]) / den)
+        L.append((m + np.log(den))[:, 0])
+    return np.concatenate(O), np.concatenate(L)
+
+
+def dense_attention(q, k, v, causal: bool, scale: float, rows=None, block: int = 128):
+    """Plain softmax attention (every key block kept), same conventions."""
+    M = q.shape[0]
+    nb = M // block
+    allk = {r: (np.arange(r + 1) if causal else np.arange(nb)) for r in range(nb)}
+    return block_sparse_attention(q, k, v, allk, block, causal, scale, rows)
+
+
+# ------------------------------------------------------------- layer wrappers
+def layer_block_scores(Qb, Kb, Hkv: int, stride: int, block: int, sigma: float,
+                       causal: bool, heads=None, rows=None, antidiagonal: bool = True):
+    """Scores for (batch, query head) pairs of bf16-bit tensors Q [B,Hq,M,C], K [B,Hkv,M,C].
+
+    Returns {(b, h): [nb, nb]}. Query head h uses KV head h // (Hq/Hkv).
+    """
+    B, Hq = Qb.shape[:2]
+    grp = Hq // Hkv
+    heads = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else heads
+    out = {}
+    for (b, h) in heads:
+        q = bf16_to_f64(Qb[b, h])
+        k = bf16_to_f64(Kb[b, h // grp])
+        out[(b, h)] = block_scores(q, k, stride, block, sigma, causal, rows, antidiagonal)
+    return out
+
+
+def layer_select(scores_by_head, tau, causal: bool, rows=None):
+    """{(b, h): {r: kept}} using tau[h]."""
+    return {(b, h): select_blocks(s, float(tau[h]), causal, rows)
+            for (b, h), s in scores_by_head.items()}
+
+
+def layer_sparse_attention(Qb, Kb, Vb, Hkv: int, kept_by_head, block: int, causal: bool,
+                           scale: float, rows=None):
+    """{(b, h): (O, lse)} for the given kept lists."""
+    Hq = Qb.shape[1]
+    grp = Hq // Hkv
+    out = {}
+    for (b, h), kept in kept_by_head.items():
+        q = bf16_to_f64(Qb[b, h])
+        k = bf16_to_f64(Kb[b, h // grp])
+        v = bf16_to_f64(Vb[b, h // grp])
+        out[(b, h)] = block_sparse_attention(q, k, v, kept, block, causal, scale, rows)
+    return out
