@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark: XAttention block-sparse prefill attention, one layer per step.
+
+One step = one pass of the whole path (score -> select -> block-sparse attention)
+over one layer of seeded synthetic input (all heads), on the stream the kernels are
+launched on. Default workload: Llama-3.1-8B-shaped GQA prefill at 128K tokens
+(32 query / 8 KV heads, head dim 128, stride 8, tau 0.9, causal).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched by torchrun, one rank per GPU): the layers are independent
+problems, so every rank runs its own layer with no collective on the data path
+(weak scaling); the reported time is the max over ranks.
+
+`--impl reference` times the CPU fp64 oracle (the only reference this method has)
+on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as sy  # noqa: E402
+
+METRIC = "128K-token prefill attention ms/layer and kept-block TFLOPS (% of BF16 peak)"
+UNIT = "ms/layer"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8b_gqa_128k", choices=sorted(sy.WORKLOADS))
+    ap.add_argument("--stride", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=sy.DEFAULT_SEED)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload_of(a):
+    w = sy.workload(a.workload)
+    return w.with_(stride=a.stride) if a.stride else w
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d["bf16_tflops_sustained"], source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# --------------------------------------------------------- CPU oracle sample
+def oracle_sample(w, Qb, Kb, Vb, tau, seconds, seed=0):
+    """Time the oracle on uniformly drawn (head, query block) units until `seconds`
+    of work are done; returns (ms per layer extrapolated by unit count, units, desc)."""
+    import oracle as orc
+    from threadpoolctl import threadpool_info
+    rng = np.random.default_rng(seed)
+    nb, grp = w.nb, w.Hq // w.Hkv
+    sig, sa = orc.default_score_scale(w.stride, w.C), 1 / math.sqrt(w.C)
+    done, t_work = 0, 0.0
+    cache = {}
+    while t_work < seconds or done < 4:
+        h, r = int(rng.integers(w.Hq)), int(rng.integers(nb))
+        if h not in cache:   # input widening is data movement, not timed
+            cache.clear()
+            cache[h] = tuple(orc.bf16_to_f64(x) for x in (Qb[0, h], Kb[0, h // grp], Vb[0, h // grp]))
+        q, k, v = cache[h]
+        t0 = time.perf_counter()
+        s = orc.block_scores(q, k, w.stride, w.block, sig, w.causal, rows=[r])
+        kept = {r: orc.select_row(s[r], r, float(tau[h]), w.causal)}
+        orc.block_sparse_attention(q, k, v, kept, w.block, w.causal, sa, rows=[r])
+        t_work += time.perf_counter() - t0
+        done += 1
+    units = w.B * w.Hq * nb
+    threads = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
+    desc = (f"{done} (head, query-block) units of the {w.name} layer drawn uniformly at random "
+            f"(score row + select + sparse attention each), {t_work:.1f} s; full-layer time "
+            f"extrapolated by unit count x{units / done:.0f}")
+    return t_work / done * units * 1e3, done, desc, max(1, threads)
+
+
+def reference_arm(a, w, rank, world):
+    """--impl reference: the CPU oracle as the timed arm, rank 0 only."""
+    if rank != 0:
+        return 0
+    Qb, Kb, Vb = sy.layer_inputs(w, a.seed)
+    tau = sy.tau_vector(w, a.seed)
+    per_step = max(2.0, min(a.cpu_seconds, 60.0 / max(1, a.steps + a.warmup)))
+    for i in range(a.warmup):
+        oracle_sample(w, Qb, Kb, Vb, tau, per_step, seed=100 + i)
+    vals, units, cores, desc = [], 0, 1, ""
+    for i in range(a.steps):
+        v, u, desc, cores = oracle_sample(w, Qb, Kb, Vb, tau, per_step, seed=i)
+        vals.append(v)
+        units += u
+    val = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": val, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.M, "C": w.C,
+            "block": w.block, "stride": w.stride, "causal": w.causal,
+            "tau": list(w.tau_range) if w.tau_range else w.tau,
+            "score_scale": "1/sqrt(stride*C)", "softmax_scale": "1/sqrt(C)",
+            "l2": "inputs larger than L2 (126 MB): Q %.2f GB, K and V %.2f GB each" % (
+                w.B * w.Hq * w.M * w.C * 2 / 1e9, w.B * w.Hkv * w.M * w.C * 2 / 1e9),
+            "parallelism": "one independent layer per GPU (no collective)"}
+
+
+# ------------------------------------------------------------ our arm
+def main():
+    a = parse()
+    w = workload_of(a)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if a.impl == "reference":
+        return reference_arm(a, w, rank, world)
+
+    import torch
+    import block_sparse_long_04_b200 as xa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # inputs: generated on the host (pinned), copied once; resident in HBM when timed
+    seed = a.seed + rank
+    Qh = torch.empty((w.B, w.Hq, w.M, w.C), dtype=torch.bfloat16).pin_memory()
+    Kh = torch.empty((w.B, w.Hkv, w.M, w.C), dtype=torch.bfloat16).pin_memory()
+    Vh = torch.empty((w.B, w.Hkv, w.M, w.C), dtype=torch.bfloat16).pin_memory()
+    views = tuple(t.view(torch.int16).numpy().view(np.uint16) for t in (Qh, Kh, Vh))
+    sy.layer_inputs(w, seed, out=views)
+    tau_np = sy.tau_vector(w, seed)
+    Q, K, V = (t.to(dev) for t in (Qh, Kh, Vh))
+    tau = torch.from_numpy(tau_np).to(dev)
+    bufs = xa.Buffers.allocate(w.B, w.Hq, w.M, w.C, w.stride, w.causal, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ss = xa.default_score_scale(w.stride, w.C)
+    sa = 1 / math.sqrt(w.C)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        xa.xattn_score(Q, K, w.stride, w.causal, ss, bufs.scores, bufs.score_ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        xa.xattn_select(bufs.scores, tau, w.causal, bufs.row_ptr, bufs.col_idx, bufs.nnz,
+                        bufs.select_ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        xa.xattn_sparse_attn(Q, K, V, bufs.row_ptr, bufs.col_idx, w.causal, sa, bufs.O,
+                             stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 5   # score 1, select 3, sparse attention 1
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if xa.xattn_get_device_error() != xa.XATTN_OK:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(a.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    total_ms = max_over_ranks(t0.elapsed_time(t1))
+    ms_step = total_ms / a.steps
+    value = total_ms / (a.steps * world * w.B)        # ms per layer, whole job
+    st_score = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    st_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    st_attn = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    nnz = int(bufs.nnz.item())
+    if xa.xattn_get_device_error() != xa.XATTN_OK:
+        raise RuntimeError("device error during the timed steps")
+    b2, C = w.block ** 2, w.C
+    kept_flops = 4.0 * b2 * C * nnz
+    cand = w.B * w.Hq * (w.nb * (w.nb + 1) // 2 if w.causal else w.nb * w.nb)
+    density = nnz / cand
+    dense_eq_flops = (2.0 if w.causal else 4.0) * w.M * w.M * C * w.Hq * w.B
+    pk = peaks()
+    attn_tflops = kept_flops / (st_attn * 1e-3) / 1e12
+    roofline = {"kernel": "sparse_attn", "bound": "tensor", "achieved": attn_tflops,
+                "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": attn_tflops / pk["bf16_sustained"],
+                "peak_source": f"{pk['source']} bf16 sustained (kernel runs inside a long step)",
+                "traffic": None,
+                "algorithmic": "4*b^2*C FLOP per kept (head, query block, key block), "
+                               "diagonal blocks counted in full"}
+    score_flops = (1.0 if w.causal else 2.0) * w.M * w.M * C * w.Hq * w.B / w.stride
+    extra = {
+        "stages_ms": {"score": st_score, "select": st_select, "sparse_attn": st_attn},
+        "density": density, "nnz": nnz,
+        "kept_block_tflops": attn_tflops,
+        "kept_block_frac_of_bf16_peak": attn_tflops / pk["bf16_sustained"],
+        "dense_equivalent_tflops": dense_eq_flops / (ms_step * 1e-3) / 1e12,
+        "score_tflops": score_flops / (st_score * 1e-3) / 1e12,
+    }
+
+    # dense baseline (the build's own dense attention), same inputs
+    if not a.no_dense:
+        Od = torch.empty_like(Q)
+        for _ in range(max(1, a.warmup)):
+            xa.xattn_dense_attn(Q, K, V, w.causal, sa, Od, stream=stream)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        d0.record(stream)
+        for _ in range(a.steps):
+            xa.xattn_dense_attn(Q, K, V, w.causal, sa, Od, stream=stream)
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_ms = max_over_ranks(d0.elapsed_time(d1)) / a.steps
+        extra["dense_attn_ms"] = dense_ms
+        extra["dense_attn_tflops"] = dense_eq_flops / (dense_ms * 1e-3) / 1e12
+        extra["speedup_vs_dense"] = dense_ms / ms_step
+        del Od
+
+    # end to end through the public API with host buffers: H2D inputs, D2H output
+    e2e = None
+    if not a.no_e2e:
+        Oh = torch.empty((w.B, w.Hq, w.M, w.C), dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            Q.copy_(Qh, non_blocking=True)
+            K.copy_(Kh, non_blocking=True)
+            V.copy_(Vh, non_blocking=True)
+            tau.copy_(torch.from_numpy(tau_np), non_blocking=False)
+            xa.xattn_prefill(Q, K, V, tau, w.stride, w.causal, bufs, stream=stream)
+            Oh.copy_(bufs.O, non_blocking=True)
+
+        for _ in range(max(1, a.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_total = max_over_ranks(e0.elapsed_time(e1))
+        h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh)) + tau_np.nbytes
+        d2h = Oh.numel() * Oh.element_size()
+        e2e = {"value": e2e_total / (a.steps * world * w.B), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del Oh
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        v, units, desc, cores = oracle_sample(w, *views, tau_np, a.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * a.steps, "clocks": clk.summary(), **extra,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

