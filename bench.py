@@ -142,7 +142,7 @@ def oracle_sample(w, Qb, Kb, Vb, tau, seconds, seed=0):
     threads = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
     desc = (f"{done} (head, query-block) units of the {w.name} layer drawn uniformly at random "
             f"(score row + select + sparse attention each), {t_work:.1f} s; full-layer time "
-            f"extrapolated by unit count x{units / done:.0f}")
+            f"extrapolated by unit count (x{units / done:.3g})")
     return t_work / done * units * 1e3, done, desc, max(1, threads)
 
 
@@ -179,8 +179,9 @@ def config_of(w):
             "block": w.block, "stride": w.stride, "causal": w.causal,
             "tau": list(w.tau_range) if w.tau_range else w.tau,
             "score_scale": "1/sqrt(stride*C)", "softmax_scale": "1/sqrt(C)",
-            "l2": "inputs larger than L2 (126 MB): Q %.2f GB, K and V %.2f GB each" % (
-                w.B * w.Hq * w.M * w.C * 2 / 1e9, w.B * w.Hkv * w.M * w.C * 2 / 1e9),
+            "l2": "no flush; inputs larger than L2 (126 MB): Q %.2f GB, K and V %.2f GB each" % (
+                w.B * w.Hq * w.M * w.C * 2 / 1e9, w.B * w.Hkv * w.M * w.C * 2 / 1e9)
+            if w.B * w.Hkv * w.M * w.C * 2 > 126e6 else "inputs fit in L2 (not a bench workload)",
             "parallelism": "one independent layer per GPU (no collective)"}
 
 

@@ -1,0 +1,318 @@
+// Block-sparse (and dense) softmax attention on the 5th-generation tensor cores.
+//
+// Sparse attention over the kept key blocks only (DuSA rebuttal, Response to
+// W3/Q1; XAttention summary, Approach). One CTA = one (batch, query head, query
+// block r) tile of 128 query rows; GQA maps query head h to KV head h/(Hq/Hkv).
+//
+// Warp roles (256 threads):
+//   warp 0, one lane  TMA producer: Q once, then K/V tiles of the kept blocks
+//                     (in list order) into a ring of kStages shared-memory stages.
+//   warp 1, one lane  MMA issuer: S = Q K^T into TMEM (128 lanes x 128 fp32 cols),
+//                     then O += P V into TMEM (128 lanes x C fp32 cols). S of block
+//                     j+1 is issued as soon as the softmax has read S of block j, so
+//                     it overlaps that softmax.
+//   warps 4-7         softmax, one query row per thread (TMEM lane = row): read the
+//                     S row, causal mask on the diagonal block, online softmax in
+//                     fp32 (base 2) with lazy rescaling (O and l are rescaled only
+//                     when the running max grows by more than 2^8), write P as bf16
+//                     into shared memory in the tensor core's 128-byte-swizzled
+//                     K-major layout, and finally normalise O out of TMEM.
+// Every wait is bounded (sm100::mbar_wait); on a timeout the CTA raises
+// XATTN_ETIMEOUT, every role stops, in-flight copies and MMAs are drained, and
+// TMEM is freed before the CTA exits.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace xattn {
+
+constexpr int kAttnTcThreads = 256;
+
+template <int C>
+struct AttnTc {
+  static constexpr int kStages = (C == 64) ? 3 : 2;
+  static constexpr int kRegion = 128 * 128;        // 128 rows x 64 bf16 (128 B) = 16 KB
+  static constexpr int kNReg = C / 64;             // regions per 128-row tile
+  static constexpr int kTile = kNReg * kRegion;    // one 128 x C bf16 tile
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kTile;
+  static constexpr int kOffV = kOffK + kStages * kTile;
+  static constexpr int kOffP = kOffV + kStages * kTile;   // 128 x 128 bf16
+  static constexpr int kOffBar = kOffP + 2 * kRegion;
+  static constexpr int kSmem = kOffBar + 256 + 1024;      // + alignment slack
+  static constexpr int kTmemCols = 256;                   // S: 0..127, O: 128..128+C-1
+};
+
+template <int C, bool DENSE>
+__global__ void __launch_bounds__(kAttnTcThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ row_ptr,
+               const int32_t* __restrict__ col_idx, int Hq, int Hkv, int M, int causal,
+               float scale_log2, bf16* __restrict__ O, float* __restrict__ lse) {
+  using L = AttnTc<C>;
+  constexpr int ST = L::kStages;
+  using namespace sm100;
+
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sQ = smem_u32(smem + L::kOffQ);
+  const uint32_t sK0 = smem_u32(smem + L::kOffK);
+  const uint32_t sV0 = smem_u32(smem + L::kOffV);
+  const uint32_t sP = smem_u32(smem + L::kOffP);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + ST;
+  uint64_t* q_full = bars + 2 * ST;
+  uint64_t* s_full = q_full + 1;
+  uint64_t* s_free = q_full + 2;
+  uint64_t* p_full = q_full + 3;
+  uint64_t* o_done = q_full + 4;
+  uint64_t* drain = q_full + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 6);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nb = M / 128;
+  const int r = nb - 1 - (int)blockIdx.x;   // longest rows first
+  const int bh = blockIdx.y;
+  const int b = bh / Hq, h = bh % Hq, kvh = h / (Hq / Hkv);
+  const size_t row = (size_t)bh * nb + r;
+  int beg, end;
+  if (DENSE) { beg = 0; end = causal ? r + 1 : nb; }
+  else { beg = row_ptr[row]; end = row_ptr[row + 1]; }
+  auto block_of = [&](int it) -> int {
+    const int c = DENSE ? it : __ldg(col_idx + it);
+    return (c < 0 || c >= nb || (causal && c > r)) ? -1 : c;
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < ST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    mbar_init(q_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 32 * 2) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(q_full, L::kTile);
+      const int yq = bh * M + r * 128;
+#pragma unroll
+      for (int g = 0; g < L::kNReg; ++g) tma_load_2d(sQ + g * L::kRegion, &tmQ, g * 64, yq, q_full);
+      const int ykv = (b * Hkv + kvh) * M;
+      int j = 0;
+      for (int it = beg; it < end; ++it) {
+        const int c = block_of(it);
+        if (c < 0) continue;
+        const int st = j % ST;
+        if (j >= ST && !mbar_wait(&kv_empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&kv_full[st], 2 * L::kTile);
+#pragma unroll
+        for (int g = 0; g < L::kNReg; ++g) {
+          tma_load_2d(sK0 + st * L::kTile + g * L::kRegion, &tmK, g * 64, ykv + c * 128, &kv_full[st]);
+          tma_load_2d(sV0 + st * L::kTile + g * L::kRegion, &tmV, g * 64, ykv + c * 128, &kv_full[st]);
+        }
+        ++j;
+      }
+      // drain: every load issued must land before the CTA may exit
+      volatile int no_abort = 0;
+      mbar_wait(q_full, 0, &no_abort);
+      for (int jj = (j > ST ? j - ST : 0); jj < j; ++jj)
+        mbar_wait(&kv_full[jj % ST], (jj / ST) & 1, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int n = 0;
+      for (int it = beg; it < end; ++it) n += block_of(it) >= 0 ? 1 : 0;
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(128, C, false, true);
+      auto issue_S = [&](int j) {
+        const int st = j % ST;
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kRegion + (kk & 3) * 32;
+          mma_f16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024),
+                     smem_desc_sw128(sK0 + st * L::kTile + off, 16, 1024), idS, kk > 0);
+        }
+        mma_commit(s_full);
+      };
+      bool ok = n > 0 && mbar_wait(q_full, 0, abort_flag);
+      if (ok) ok = mbar_wait(&kv_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_S(0);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n) {
+          ok = mbar_wait(&kv_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag) &&
+               mbar_wait(s_free, j & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_S(j + 1);
+        }
+        if (!(ok = mbar_wait(p_full, j & 1, abort_flag))) break;
+        tc_fence_after();
+        const int st = j % ST;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a_off = (kk >> 2) * L::kRegion + (kk & 3) * 32;
+          mma_f16_ss(tO, smem_desc_sw128(sP + a_off, 16, 1024),
+                     smem_desc_sw128(sV0 + st * L::kTile + kk * 2048, L::kRegion, 1024), idPV,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(o_done);
+        mma_commit(&kv_empty[st]);
+      }
+      // drain: all MMAs issued by this thread complete before TMEM is freed
+      mma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- softmax
+    const int q_row = (warp & 3) * 32 + lane;          // row within the query block
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float m = kNegInf, l = 0.f;
+    int j = 0;
+    bool ok = true;
+    float s[128];
+    for (int it = beg; it < end; ++it) {
+      const int c = block_of(it);
+      if (c < 0) continue;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + lane_off + q * 32, s + q * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+
+      const bool diag = causal && (c == r);
+      float mx = kNegInf;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        float x = s[i] * scale_log2;
+        x = (diag && i > q_row) ? kNegInf : x;
+        s[i] = x;
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m, mx);
+      float corr = 1.f;
+      bool resc = false;
+      if (j == 0) {
+        m = m_new;
+      } else if (m_new > m + 8.f) {
+        corr = ex2(m - m_new);
+        m = m_new;
+        resc = true;
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        s[i] = ex2(s[i] - m);
+        rs += s[i];
+      }
+      l = l * corr + rs;
+
+      // PV of the previous block must be complete: P buffer free, O stable
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int q = 0; q < C / 32; ++q) {
+          float o[32];
+          tmem_ld32(tO + lane_off + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= corr;
+          tmem_st32(tO + lane_off + q * 32, o);
+        }
+        tmem_wait_st();
+      }
+      // P row -> shared memory, 128-byte swizzled K-major (two 64-key regions)
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        uint4 v;
+        v.x = pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]);
+        v.y = pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]);
+        v.z = pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]);
+        v.w = pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]);
+        const uint32_t addr = sP + (ch >> 3) * L::kRegion + q_row * 128 + (((ch & 7) ^ (q_row & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                     "r"(v.z), "r"(v.w) : "memory");
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      ++j;
+    }
+
+    // epilogue: O / l -> bf16 global; lse = (m + log2 l) ln 2
+    bf16* orow = O + ((size_t)bh * M + (size_t)r * 128 + q_row) * C;
+    if (ok && j > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int q = 0; q < C / 32; ++q) {
+          float o[32];
+          tmem_ld32(tO + lane_off + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(o[i + 0] * inv, o[i + 1] * inv);
+            v.y = pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv);
+            v.z = pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv);
+            v.w = pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
+          }
+        }
+        if (lse != nullptr)
+          lse[(size_t)bh * M + (size_t)r * 128 + q_row] = l > 0.f ? (m + lg2(l)) * kLn2 : kNegInf;
+      }
+    } else if (ok && j == 0) {
+      const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < C; i += 8) *reinterpret_cast<uint4*>(orow + i) = z;
+      if (lse != nullptr) lse[(size_t)bh * M + (size_t)r * 128 + q_row] = kNegInf;
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace xattn

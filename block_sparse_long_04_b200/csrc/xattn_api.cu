@@ -2,9 +2,12 @@
 // The contract of every entry point is documented in include/xattn.h.
 #include "xattn.h"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "attn_mma.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "score_mma.cuh"
 #include "select.cuh"
@@ -81,6 +84,53 @@ int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int 
   return XATTN_EUNSUPPORTED;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows, C] bf16 matrix with 128-row x 64-column boxes, 128-byte
+// swizzle (the layout the tensor core's SW128 descriptors read).
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int C) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)C * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int C, bool DENSE>
+int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
+                   const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
+                   bf16* O, float* lse, cudaStream_t st) {
+  auto kern = attn_tc_kernel<C, DENSE>;
+  constexpr int smem = AttnTc<C>::kSmem;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_tile_map(&mq, Q, (uint64_t)B * Hq * M, C) ||
+      !make_tile_map(&mk, K, (uint64_t)B * Hkv * M, C) ||
+      !make_tile_map(&mv, V, (uint64_t)B * Hkv * M, C))
+    return XATTN_ECUDA;
+  dim3 grid(M / 128, B * Hq);
+  kern<<<grid, kAttnTcThreads, smem, st>>>(mq, mk, mv, row_ptr, col_idx, Hq, Hkv, M, causal,
+                                           scale * kLog2e, O, lse);
+  return launch_status();
+}
+
 template <int C, bool DENSE>
 int launch_attn(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
                 const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
@@ -112,11 +162,19 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_
   auto v = static_cast<const bf16*>(V);
   auto o = static_cast<bf16*>(O);
   cudaStream_t st = as_stream(stream);
+#ifndef XATTN_TC_ATTN
   if (C == 64)
     return launch_attn<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                   softmax_scale, o, lse, st);
   return launch_attn<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                  softmax_scale, o, lse, st);
+#else
+  if (C == 64)
+    return launch_attn_tc<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
+                                     softmax_scale, o, lse, st);
+  return launch_attn_tc<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
+                                    softmax_scale, o, lse, st);
+#endif
 }
 
 }  // namespace
