@@ -42,6 +42,7 @@ SIGNATURES = {
     "xattn_sparse_attn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "xattn_dense_attn": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "xattn_get_device_error": (_I, [_P]),
+    "xattn_select_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _Z, _P, _P]),
 }
 
 
@@ -138,6 +139,21 @@ def xattn_select(scores, tau, causal: bool, row_ptr, col_idx, nnz, workspace, st
                            _ptr(col_idx), col_idx.numel(), _ptr(nnz), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "xattn_select")
+
+
+def xattn_select_noalloc(scores, tau, causal: bool, row_ptr, col_idx, nnz, stream=None) -> None:
+    """xattn_select without a workspace, for callers that cannot allocate device
+    memory while this step runs: the library keeps a fixed scratch array of
+    XATTN_SELECT_NOALLOC_MAX_ROWS rows per device. Calls that overlap on the GPU
+    race on that array, so issue them on one stream."""
+    _dev(scores, tau, row_ptr, col_idx, nnz)
+    B, Hq, nb, _ = scores.shape
+    rc = _lib.xattn_select_noalloc(_ptr(scores), _ptr(tau), B, Hq, nb, int(causal), _ptr(row_ptr),
+                                   _ptr(col_idx), col_idx.numel(), _ptr(nnz), _stream(stream))
+    _check(rc, "xattn_select_noalloc")
+
+
+XATTN_SELECT_NOALLOC_MAX_ROWS = 262144
 
 
 def xattn_sparse_attn(Q, K, V, row_ptr, col_idx, causal: bool, softmax_scale: float, O,

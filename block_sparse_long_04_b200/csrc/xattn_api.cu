@@ -273,6 +273,60 @@ int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, i
   return launch_status();
 }
 
+// ---- selection without a caller workspace -------------------------------
+// The per-row scratch of xattn_select_noalloc: a fixed device array, so that the
+// entry point needs no workspace and calls no allocator.
+static __device__ __align__(256) SelCut g_select_scratch[XATTN_SELECT_NOALLOC_MAX_ROWS];
+
+// Device address of g_select_scratch for the current device. The name is a
+// host-side stand-in, not a device address, so it is looked up once per device
+// (with that device current) and cached.
+static SelCut* select_scratch_on_current_device() {
+  static SelCut* cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SelCut* p = __atomic_load_n(&cached[dev], __ATOMIC_ACQUIRE);
+  if (p != nullptr) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_select_scratch) != cudaSuccess || addr == nullptr)
+    return nullptr;
+  __atomic_store_n(&cached[dev], static_cast<SelCut*>(addr), __ATOMIC_RELEASE);
+  return static_cast<SelCut*>(addr);
+}
+
+int xattn_select_noalloc(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
+                         int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
+                         void* stream) {
+  if (B < 0 || Hq < 0 || nb < 0) return XATTN_EINVAL;
+  const long long rows = (long long)B * Hq * nb;
+  if (nb > kSelMaxNb || rows > XATTN_SELECT_NOALLOC_MAX_ROWS) return XATTN_EUNSUPPORTED;
+  const long long worst = causal ? rows * (nb + 1) / 2 : rows * nb;
+  if (worst >= (1LL << 31)) return XATTN_EUNSUPPORTED;
+  if (!row_ptr || !nnz) return XATTN_EINVAL;
+  cudaStream_t st = as_stream(stream);
+  if (rows == 0) {
+    if (cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    return XATTN_OK;
+  }
+  if (!scores || !tau || !col_idx) return XATTN_EINVAL;
+  SelCut* cuts = select_scratch_on_current_device();
+  if (cuts == nullptr) return XATTN_ECUDA;
+  int P = 1;
+  while (P < nb) P <<= 1;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
+  select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, tau, Hq, nb,
+                                                                  causal ? 1 : 0, cuts);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
+  select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
+                                                              row_ptr, col_idx);
+  return launch_status();
+}
+
 int xattn_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                       const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
                       int causal, float softmax_scale, void* O, float* lse, void* stream) {

@@ -138,6 +138,41 @@ XATTN_API int xattn_select(const float* scores, const float* tau, int B, int Hq,
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Largest number of selection rows (B*Hq*nb) that xattn_select_noalloc takes.
+ */
+#define XATTN_SELECT_NOALLOC_MAX_ROWS 262144
+
+/*
+ * xattn_select_noalloc - the same selection as xattn_select, for callers that
+ * cannot hand the library a workspace. This is a library convenience; the
+ * pages describe no counterpart.
+ *
+ * Some callers cannot allocate device memory when they run this step: a host
+ * framework that owns all device memory and forbids allocation inside its
+ * execute callbacks (plugins, custom operators with a fixed memory plan), or a
+ * latency-critical caller that cannot afford the device-wide synchronisation a
+ * cudaMalloc may bring. This entry point takes no workspace and calls no
+ * allocator: its per-row scratch (12 bytes per row) lives in a fixed array
+ * inside the library, XATTN_SELECT_NOALLOC_MAX_ROWS rows (3 MiB), which every
+ * GPU that loads the library holds until the process exits.
+ *
+ * Arguments, outputs and capacity behaviour are those of xattn_select. The
+ * caller still provides every input and output buffer.
+ *   - B*Hq*nb above XATTN_SELECT_NOALLOC_MAX_ROWS returns XATTN_EUNSUPPORTED
+ *     before any launch.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one scratch array, and calls whose work
+ *     overlaps on the GPU (different streams, or different host threads) race
+ *     on it. Serialise them, e.g. issue them on one stream. The scratch keeps
+ *     the last call's contents; each call overwrites every row it reads.
+ */
+XATTN_API int xattn_select_noalloc(const float* scores, const float* tau, int B, int Hq, int nb,
+                                   int causal, int32_t* row_ptr, int32_t* col_idx,
+                                   size_t col_capacity, int32_t* nnz, void* stream);
+
+/*
  * xattn_sparse_attn - block-sparse softmax attention [DuSA-W3, XA-app].
  *
  * For query token i of block r of head h (KV head h/(Hq/Hkv)):

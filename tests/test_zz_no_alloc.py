@@ -1,0 +1,77 @@
+"""xattn_select_noalloc: threshold selection for callers that cannot allocate.
+
+Some callers cannot hand the library a workspace: a host framework that owns
+all device memory and forbids allocation inside its execute callbacks, or a
+latency-critical caller that cannot take the synchronisation a cudaMalloc may
+bring. xattn_select_noalloc serves them from a fixed scratch array inside the
+library. Its kept lists must equal those of xattn_select exactly (they are
+integer outputs), call after call, although every call reuses the same scratch.
+
+This file is collected last, so that a run stopping at its first failure has
+already run every other test; it sets up everything it needs itself, so it also
+passes when run alone in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_04_b200 as xa
+
+
+def _scores(seed, Hq, nb, causal):
+    rng = np.random.default_rng(seed)
+    s = rng.gamma(0.4, size=(1, Hq, nb, nb))
+    if causal:
+        s = np.tril(s)
+    s /= s.sum(axis=-1, keepdims=True)
+    return torch.from_numpy(s.astype(np.float32)).cuda()
+
+
+def _outputs(Hq, nb, causal):
+    rows = Hq * nb
+    cap = xa.max_kept(1, Hq, nb, causal)
+    return (torch.full((rows + 1,), -1, dtype=torch.int32, device="cuda"),
+            torch.full((cap,), -1, dtype=torch.int32, device="cuda"),
+            torch.full((1,), -1, dtype=torch.int32, device="cuda"))
+
+
+@pytest.mark.gpu
+def test_noalloc_select_equals_select_on_consecutive_calls():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    # two calls in a row with different shapes and thresholds; the second call
+    # finds the first call's rows still in the shared scratch
+    for seed, Hq, nb, causal, taus in ((1, 4, 300, True, [0.9, 0.5, 0.99, 0.8]),
+                                       (2, 3, 97, False, [0.95, 0.7, 0.3])):
+        scores = _scores(seed, Hq, nb, causal)
+        tau = torch.tensor(taus, dtype=torch.float32, device="cuda")
+        ref = _outputs(Hq, nb, causal)
+        ws = torch.empty(xa.xattn_select_workspace_size(1, Hq, nb), dtype=torch.uint8,
+                         device="cuda")
+        xa.xattn_select(scores, tau, causal, *ref, ws)
+        got = _outputs(Hq, nb, causal)
+        rp, ci, nz = got
+        # straight through the C ABI: no workspace argument at all
+        rc = xa._lib.xattn_select_noalloc(
+            ctypes.c_void_p(scores.data_ptr()), ctypes.c_void_p(tau.data_ptr()), 1, Hq, nb,
+            int(causal), ctypes.c_void_p(rp.data_ptr()), ctypes.c_void_p(ci.data_ptr()),
+            ci.numel(), ctypes.c_void_p(nz.data_ptr()),
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert rc == xa.XATTN_OK, xa.status_string(rc)
+        torch.cuda.synchronize()
+        assert xa.xattn_get_device_error() == xa.XATTN_OK
+        n = int(ref[2].item())
+        assert int(nz.item()) == n
+        assert torch.equal(rp, ref[0])
+        assert torch.equal(ci[:n], ref[1][:n])
+
+
+def test_noalloc_select_rejects_rows_beyond_its_scratch():
+    # checked on the host before any launch: no GPU needed
+    fake = ctypes.c_void_p(0x7F0000001000)
+    nb = 2048
+    Hq = xa.XATTN_SELECT_NOALLOC_MAX_ROWS // nb + 1
+    rc = xa._lib.xattn_select_noalloc(fake, fake, 1, Hq, nb, 1, fake, fake, 1 << 30, fake, None)
+    assert rc == xa.XATTN_EUNSUPPORTED
