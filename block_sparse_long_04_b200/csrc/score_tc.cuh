@@ -1,0 +1,237 @@
+// Strided antidiagonal block scoring on the 5th-generation tensor cores.
+//
+// One CTA owns 128 reshaped query rows i' of one (batch, query head) and sweeps
+// the reshaped key columns j' in tiles of BN (only tiles reaching j' <= i' when
+// causal). The reshaped rows (DuSA rebuttal, Response to Q2) are never built:
+// Q is read through a 2-D TMA map over [B*Hq*M/S, S*C] and K through one over
+// [B*Hkv*M/S, S*C]; for stride slot s the query chunk is taken at column
+// (S-1-s)*C (rows reversed inside each stride group) and the key chunk at s*C, so
+// every dot product is an S-long lower-left -> upper-right antidiagonal of q k^T
+// (XAttention abstract). The reduction over S*C runs in 64-element chunks
+// through a ring of shared-memory stages; each chunk is four M=128 x N=BN x K=16
+// tcgen05 MMAs into a TMEM accumulator, double-buffered so that the epilogue of
+// one column tile overlaps the MMAs of the next.
+//
+// Warp roles (256 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA
+// issuer (warp 1 also owns the TMEM allocation), warps 4-7 = epilogue, one
+// reshaped row per thread (TMEM lane = row).
+//
+// Epilogue (row softmax + block summation, XAttention summary, Approach): for
+// every key block of g = 128/S columns the thread forms the block's base-2
+// log-sum-exp ell[i', c] from its TMEM row, updates the row's running LSE, and
+// writes ell to the workspace. After the sweep the same threads re-read their
+// CTA's ell values (L2-resident) and write
+//   scores[r, c] = (1/g) sum_{i' in r} 2^(ell[i', c] - LSE[i']).
+// The (M/S)^2 logits are never stored. Waits are bounded as in attn_tc.cuh.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace xattn {
+
+constexpr int kScoreTcThreads = 256;
+
+template <int BN>
+struct ScoreTc {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kQBytes = 128 * 128;              // 128 rows x 64 bf16
+  static constexpr int kKBytes = BN * 128;               // BN rows x 64 bf16
+  static constexpr int kStageBytes = kQBytes + kKBytes;
+  static constexpr int kOffBar = kStages * kStageBytes;
+  static constexpr int kOffLse = kOffBar + 256;
+  static constexpr int kSmem = kOffLse + 128 * 4 + 1024;
+  static constexpr int kTmemCols = 2 * BN;
+};
+
+template <int C, int G, int BN>
+__global__ void __launch_bounds__(kScoreTcThreads, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                int Hq, int Hkv, int M, int causal, float scale_log2, float* __restrict__ part,
+                float* __restrict__ lse_ws, float* __restrict__ scores) {
+  using L = ScoreTc<BN>;
+  constexpr int ST = L::kStages;
+  constexpr int S = 128 / G;
+  constexpr int NCH = S * C / 64;       // 64-wide chunks of the reshaped width
+  using namespace sm100;
+
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;                 // [ST]
+  uint64_t* empty = bars + ST;           // [ST]
+  uint64_t* acc_full = bars + 2 * ST;    // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* drain = acc_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* lse_s = reinterpret_cast<float*>(smem + L::kOffLse);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rp = M / S;
+  const int nb = M / 128;
+  const int RT = (rp + 127) / 128;
+  const int t = causal ? (RT - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / Hq, h = bh % Hq, kvh = h / (Hq / Hkv);
+  const int i0 = t * 128;
+  // column tiles: causal needs columns up to i0 + 127
+  const int njt = causal ? min((i0 + 127) / BN + 1, (rp + BN - 1) / BN) : (rp + BN - 1) / BN;
+  const int total = njt * NCH;
+
+  if (tid == 0) {
+    for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 64) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const int yq = bh * rp + i0;
+      const int yk0 = (b * Hkv + kvh) * rp;
+      int it = 0;
+      for (; it < total; ++it) {
+        const int st = it % ST;
+        if (it >= ST && !mbar_wait(&empty[st], ((it / ST) - 1) & 1, abort_flag)) break;
+        const int jt = it / NCH, q = it % NCH;
+        const int s = (q * 64) / C, d0 = (q * 64) % C;
+        mbar_expect_tx(&full[st], L::kStageBytes);
+        const uint32_t dst = sbase + st * L::kStageBytes;
+        tma_load_2d(dst, &tmQ, (S - 1 - s) * C + d0, yq, &full[st]);
+        tma_load_2d(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, &full[st]);
+      }
+      volatile int no_abort = 0;
+      for (int jj = (it > ST ? it - ST : 0); jj < it; ++jj)
+        mbar_wait(&full[jj % ST], (jj / ST) & 1, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      bool ok = true;
+      for (int it = 0; ok && it < total; ++it) {
+        const int st = it % ST;
+        const int jt = it / NCH, q = it % NCH;
+        const int buf = jt & 1;
+        if (q == 0 && jt >= 2) {
+          if (!(ok = mbar_wait(&acc_empty[buf], ((jt / 2) - 1) & 1, abort_flag))) break;
+        }
+        if (!(ok = mbar_wait(&full[st], (it / ST) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t a0 = sbase + st * L::kStageBytes;
+        const uint32_t b0 = a0 + L::kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16_ss(tmem + buf * BN, smem_desc_sw128(a0 + kk * 32, 16, 1024),
+                     smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc, (q > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&empty[st]);
+        if (q == NCH - 1) mma_commit(&acc_full[buf]);
+      }
+      mma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- epilogue
+    const int rl = (warp & 3) * 32 + lane;     // row within the tile
+    const int ip = i0 + rl;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float m_run = kNegInf, l_run = 0.f;
+    bool ok = true;
+    for (int jt = 0; jt < njt; ++jt) {
+      const int buf = jt & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (jt / 2) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int half = 0; half < BN / 128; ++half) {
+        float v[128];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          tmem_ld32(tmem + lane_off + buf * BN + half * 128 + q4 * 32, v + q4 * 32);
+        tmem_wait_ld();
+        if (half == BN / 128 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        const int j0 = jt * BN + half * 128;
+#pragma unroll
+        for (int kb = 0; kb < 128 / G; ++kb) {
+          float vmax = kNegInf;
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            const int jp = j0 + kb * G + i;
+            float x = v[kb * G + i] * scale_log2;
+            x = (jp < rp && (!causal || jp <= ip)) ? x : kNegInf;
+            v[kb * G + i] = x;
+            vmax = fmaxf(vmax, x);
+          }
+          if (vmax != kNegInf) {
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < G; ++i) sum += ex2(v[kb * G + i] - vmax);
+            const float ell = vmax + lg2(sum);
+            const float mn = fmaxf(m_run, ell);
+            l_run = l_run * ex2(m_run - mn) + ex2(ell - mn);
+            m_run = mn;
+            if (ip < rp) part[((size_t)bh * rp + ip) * nb + (j0 / G + kb)] = ell;
+          }
+        }
+      }
+    }
+
+    // ---- finalize among the 128 epilogue threads (named barrier 1) ----
+    if (ok) {
+      const float L_row = (l_run > 0.f) ? m_run + lg2(l_run) : kNegInf;
+      lse_s[rl] = L_row;
+      if (ip < rp) lse_ws[(size_t)bh * rp + ip] = L_row;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && !*abort_flag) {
+      const int et = tid - 128;
+      const float inv_g = 1.f / (float)G;
+      for (int k = 0; k < 128 / G; ++k) {
+        const int r = i0 / G + k;
+        if (r >= nb) break;
+        const int ncand = causal ? r + 1 : nb;
+        float* srow = scores + ((size_t)bh * nb + r) * nb;
+        const float* pr0 = part + ((size_t)bh * rp + (size_t)r * G) * nb;
+        for (int c = et; c < nb; c += 128) {
+          float acc = 0.f;
+          if (c < ncand) {
+#pragma unroll 4
+            for (int i = 0; i < G; ++i) acc += ex2(pr0[(size_t)i * nb + c] - lse_s[r * G + i - i0]);
+            acc *= inv_g;
+          }
+          srow[c] = acc;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace xattn

@@ -6,10 +6,10 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
-#include "attn_mma.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "score_mma.cuh"
+#include "score_tc.cuh"
 #include "select.cuh"
 
 using namespace xattn;
@@ -36,6 +36,35 @@ int ensure_smem_limit(F* kern, int bytes, unsigned long long* done_mask) {
 
 inline int launch_status() {
   return cudaGetLastError() == cudaSuccess ? XATTN_OK : XATTN_ECUDA;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows, width] bf16 matrix with box_rows x 64-column boxes and
+// 128-byte swizzle (the layout the tensor core's SW128 descriptors read).
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int width,
+                   int box_rows = 128) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)width * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool stride_supported(int stride) {
@@ -70,10 +99,39 @@ int launch_score(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, in
   return launch_status();
 }
 
+template <int C, int G>
+int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
+                    float scale, float* scores, float* part, float* lse_ws, cudaStream_t st) {
+  constexpr int BN = 128;
+  auto kern = score_tc_kernel<C, G, BN>;
+  constexpr int smem = ScoreTc<BN>::kSmem;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
+  const int S = 128 / G;
+  const int rp = M / S;
+  CUtensorMap mq, mk;
+  if (!make_tile_map(&mq, Q, (uint64_t)B * Hq * rp, S * C, 128) ||
+      !make_tile_map(&mk, K, (uint64_t)B * Hkv * rp, S * C, BN))
+    return XATTN_ECUDA;
+  dim3 grid((rp + 127) / 128, B * Hq);
+  kern<<<grid, kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, scale * kLog2e, part,
+                                            lse_ws, scores);
+  return launch_status();
+}
+
 template <int C>
 int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
                    int causal, float scale, float* scores, float* part, float* lse_ws,
                    cudaStream_t st) {
+#ifdef XATTN_TC_SCORE
+  switch (stride) {
+    case 1: return launch_score_tc<C, 128>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 2: return launch_score_tc<C, 64>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 4: return launch_score_tc<C, 32>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 8: return launch_score_tc<C, 16>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 16: return launch_score_tc<C, 8>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+  }
+#else
   switch (stride) {
     case 1: return launch_score<C, 128>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
     case 2: return launch_score<C, 64>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
@@ -81,35 +139,8 @@ int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int 
     case 8: return launch_score<C, 16>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
     case 16: return launch_score<C, 8>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
   }
+#endif
   return XATTN_EUNSUPPORTED;
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2-D map over a [rows, C] bf16 matrix with 128-row x 64-column boxes, 128-byte
-// swizzle (the layout the tensor core's SW128 descriptors read).
-bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int C) {
-  auto enc = tensor_map_encoder();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)C * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int C, bool DENSE>
@@ -131,20 +162,6 @@ int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* r
   return launch_status();
 }
 
-template <int C, bool DENSE>
-int launch_attn(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
-                const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
-                bf16* O, float* lse, cudaStream_t st) {
-  auto kern = attn_mma_kernel<C, DENSE>;
-  constexpr int smem = attn_smem_bytes<C>();
-  static unsigned long long done = 0;
-  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
-  dim3 grid(M / 128, B * Hq);
-  kern<<<grid, kAttnThreads, smem, st>>>(Q, K, V, row_ptr, col_idx, Hq, Hkv, M, causal,
-                                         scale * kLog2e, O, lse);
-  return launch_status();
-}
-
 template <bool DENSE>
 int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                 const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
@@ -162,19 +179,11 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_
   auto v = static_cast<const bf16*>(V);
   auto o = static_cast<bf16*>(O);
   cudaStream_t st = as_stream(stream);
-#ifndef XATTN_TC_ATTN
-  if (C == 64)
-    return launch_attn<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
-                                  softmax_scale, o, lse, st);
-  return launch_attn<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
-                                 softmax_scale, o, lse, st);
-#else
   if (C == 64)
     return launch_attn_tc<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                      softmax_scale, o, lse, st);
   return launch_attn_tc<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                     softmax_scale, o, lse, st);
-#endif
 }
 
 }  // namespace
