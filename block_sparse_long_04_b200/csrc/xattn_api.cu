@@ -7,8 +7,8 @@
 #include <cuda_runtime.h>
 
 #include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 #include "common.cuh"
-#include "score_mma.cuh"
 #include "score_tc.cuh"
 #include "select.cuh"
 
@@ -85,21 +85,6 @@ int check_shape(int B, int Hq, int Hkv, int M, int C, int block) {
 }
 
 template <int C, int G>
-int launch_score(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
-                 float scale, float* scores, float* part, float* lse_ws, cudaStream_t st) {
-  auto kern = score_mma_kernel<C, G>;
-  static unsigned long long done = 0;
-  if (ensure_smem_limit(kern, kScoreSmem, &done) != XATTN_OK) return XATTN_ECUDA;
-  const int S = 128 / G;
-  const int rp = M / S;
-  const int RT = (rp + kScoreTile - 1) / kScoreTile;
-  dim3 grid(RT, B * Hq);
-  kern<<<grid, kScoreThreads, kScoreSmem, st>>>(Q, K, Hq, Hkv, M, causal, scale * kLog2e, part,
-                                                lse_ws, scores);
-  return launch_status();
-}
-
-template <int C, int G>
 int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
                     float scale, float* scores, float* part, float* lse_ws, cudaStream_t st) {
   constexpr int BN = 128;
@@ -123,7 +108,6 @@ template <int C>
 int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
                    int causal, float scale, float* scores, float* part, float* lse_ws,
                    cudaStream_t st) {
-#ifdef XATTN_TC_SCORE
   switch (stride) {
     case 1: return launch_score_tc<C, 128>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
     case 2: return launch_score_tc<C, 64>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
@@ -131,15 +115,6 @@ int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int 
     case 8: return launch_score_tc<C, 16>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
     case 16: return launch_score_tc<C, 8>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
   }
-#else
-  switch (stride) {
-    case 1: return launch_score<C, 128>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 2: return launch_score<C, 64>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 4: return launch_score<C, 32>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 8: return launch_score<C, 16>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 16: return launch_score<C, 8>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-  }
-#endif
   return XATTN_EUNSUPPORTED;
 }
 
@@ -162,6 +137,25 @@ int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* r
   return launch_status();
 }
 
+template <int C, bool DENSE>
+int launch_attn_tc2(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
+                    const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
+                    bf16* O, float* lse, cudaStream_t st) {
+  auto kern = attn_tc2_kernel<C, DENSE>;
+  constexpr int smem = AttnTc2<C>::kSmem;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_tile_map(&mq, Q, (uint64_t)B * Hq * M, C) ||
+      !make_tile_map(&mk, K, (uint64_t)B * Hkv * M, C) ||
+      !make_tile_map(&mv, V, (uint64_t)B * Hkv * M, C))
+    return XATTN_ECUDA;
+  dim3 grid(M / 128, B * Hq);
+  kern<<<grid, kAttnTc2Threads, smem, st>>>(mq, mk, mv, row_ptr, col_idx, Hq, Hkv, M, causal,
+                                            scale * kLog2e, O, lse);
+  return launch_status();
+}
+
 template <bool DENSE>
 int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                 const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
@@ -179,11 +173,19 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_
   auto v = static_cast<const bf16*>(V);
   auto o = static_cast<bf16*>(O);
   cudaStream_t st = as_stream(stream);
+#ifndef XATTN_ATTN_SPLIT
   if (C == 64)
     return launch_attn_tc<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                      softmax_scale, o, lse, st);
   return launch_attn_tc<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                     softmax_scale, o, lse, st);
+#else
+  if (C == 64)
+    return launch_attn_tc2<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
+                                      softmax_scale, o, lse, st);
+  return launch_attn_tc2<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
+                                     softmax_scale, o, lse, st);
+#endif
 }
 
 }  // namespace
@@ -226,7 +228,7 @@ int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int
   const size_t need = xattn_score_workspace_size(B, Hq, M, stride, block);
   if (workspace_bytes < need) return XATTN_EINVAL;
   const int rp = M / stride;
-  if ((rp + kScoreTile - 1) / kScoreTile > (1 << 30)) return XATTN_EUNSUPPORTED;
+  if ((rp + 127) / 128 > (1 << 30)) return XATTN_EUNSUPPORTED;
   float* part = static_cast<float*>(workspace);
   float* lse_ws = part + (size_t)B * Hq * rp * (M / block);
   auto q = static_cast<const bf16*>(Q);
