@@ -43,7 +43,12 @@ SIGNATURES = {
     "xattn_dense_attn": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]),
     "xattn_get_device_error": (_I, [_P]),
     "xattn_select_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _Z, _P, _P]),
+    "xattn_score_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _Z, _P]),
+    "xattn_select_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
 }
+
+XATTN_PATTERN_ANTIDIAGONAL, XATTN_PATTERN_DIAGONAL = 0, 1
+XATTN_SELECT_THRESHOLD, XATTN_SELECT_TOPK, XATTN_SELECT_RATIO = 0, 1, 2
 
 
 class XAttnError(RuntimeError):
@@ -129,6 +134,32 @@ def xattn_score(Q, K, stride: int, causal: bool, score_scale: float, scores, wor
                           float(score_scale), _ptr(scores), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "xattn_score")
+
+
+def xattn_score_ex(Q, K, stride: int, causal: bool, pattern: int, score_scale: float, scores,
+                   workspace, block: int = 128, stream=None) -> None:
+    """xattn_score with a pattern: XATTN_PATTERN_ANTIDIAGONAL or XATTN_PATTERN_DIAGONAL."""
+    _dev(Q, K, scores, workspace)
+    _bf16(Q, K)
+    B, Hq, M, C = Q.shape
+    Hkv = K.shape[1]
+    rc = _lib.xattn_score_ex(_ptr(Q), _ptr(K), B, Hq, Hkv, M, C, stride, block, int(causal),
+                             int(pattern), float(score_scale), _ptr(scores), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "xattn_score_ex")
+
+
+def xattn_select_ex(scores, param, rule: int, causal: bool, row_ptr, col_idx, nnz, workspace,
+                    stream=None) -> None:
+    """Selection by XATTN_SELECT_THRESHOLD (param = tau), XATTN_SELECT_TOPK (param = k)
+    or XATTN_SELECT_RATIO (param = fraction of the candidates)."""
+    _dev(scores, param, row_ptr, col_idx, nnz, workspace)
+    B, Hq, nb, _ = scores.shape
+    rc = _lib.xattn_select_ex(_ptr(scores), _ptr(param), int(rule), B, Hq, nb, int(causal),
+                              _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(nnz),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(rc, "xattn_select_ex")
 
 
 def xattn_select(scores, tau, causal: bool, row_ptr, col_idx, nnz, workspace, stream=None) -> None:

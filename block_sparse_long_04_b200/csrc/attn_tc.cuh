@@ -209,16 +209,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
 
-      const bool diag = causal && (c == r);
-      float mx = kNegInf;
+      // row max of the raw logits (the scale is positive); masked keys of the
+      // diagonal block are set to -inf first, on the diagonal block only
+      if (causal && c == r) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float x = s[i] * scale_log2;
-        x = (diag && i > q_row) ? kNegInf : x;
-        s[i] = x;
-        mx = fmaxf(mx, x);
+        for (int i = 0; i < 128; ++i) s[i] = (i > q_row) ? kNegInf : s[i];
       }
-      const float m_new = fmaxf(m, mx);
+      // eight independent partial maxima / sums keep the reductions off one
+      // 128-long dependency chain
+      float pm[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) pm[k] = s[k];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      const float m_new = fmaxf(m, mx * scale_log2);
       float corr = 1.f;
       bool resc = false;
       if (j == 0) {
@@ -228,12 +234,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         m = m_new;
         resc = true;
       }
-      float rs = 0.f;
+      const float neg_m = -m;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 128; ++i) {
-        s[i] = ex2(s[i] - m);
-        rs += s[i];
+        s[i] = ex2(fmaf(s[i], scale_log2, neg_m));
+        ps[i & 7] += s[i];
       }
+      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l = l * corr + rs;
 
       // PV of the previous block must be complete: P buffer free, O stable

@@ -7,7 +7,10 @@
 // [B*Hkv*M/S, S*C]; for stride slot s the query chunk is taken at column
 // (S-1-s)*C (rows reversed inside each stride group) and the key chunk at s*C, so
 // every dot product is an S-long lower-left -> upper-right antidiagonal of q k^T
-// (XAttention abstract). The reduction over S*C runs in 64-element chunks
+// (XAttention abstract). With `diagonal` set, the query chunk is taken at s*C
+// instead, which sums the tile's main diagonal: the diagonal-pattern variant the
+// DuSA rebuttal (Response to Q2) and the XAttention ablation compare against.
+// The reduction over S*C runs in 64-element chunks
 // through a ring of shared-memory stages; each chunk is four M=128 x N=BN x K=16
 // tcgen05 MMAs into a TMEM accumulator, double-buffered so that the epilogue of
 // one column tile overlaps the MMAs of the next.
@@ -46,8 +49,8 @@ struct ScoreTc {
 template <int C, int G, int BN>
 __global__ void __launch_bounds__(kScoreTcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                int Hq, int Hkv, int M, int causal, float scale_log2, float* __restrict__ part,
-                float* __restrict__ lse_ws, float* __restrict__ scores) {
+                int Hq, int Hkv, int M, int causal, int diagonal, float scale_log2,
+                float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores) {
   using L = ScoreTc<BN>;
   constexpr int ST = L::kStages;
   constexpr int S = 128 / G;
@@ -112,7 +115,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int s = (q * 64) / C, d0 = (q * 64) % C;
         mbar_expect_tx(&full[st], L::kStageBytes);
         const uint32_t dst = sbase + st * L::kStageBytes;
-        tma_load_2d(dst, &tmQ, (S - 1 - s) * C + d0, yq, &full[st]);
+        // antidiagonal: query rows reversed inside the stride group; diagonal: forward
+        tma_load_2d(dst, &tmQ, (diagonal ? s : S - 1 - s) * C + d0, yq, &full[st]);
         tma_load_2d(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, &full[st]);
       }
       volatile int no_abort = 0;

@@ -21,6 +21,13 @@
 namespace xattn {
 
 constexpr int kSelThreads = 256;
+
+// How the cut of a sorted row is placed.
+enum SelRule : int {
+  kSelThreshold = 0,   // shortest prefix whose cumulative score reaches param (tau)
+  kSelTopK = 1,        // the floor(param) highest-ranked candidates (at least one)
+  kSelRatio = 2,       // ceil(param * candidates) highest-ranked, taken in fp64
+};
 constexpr int kSelMaxNb = 8192;   // candidates per row held in shared memory
 
 struct SelCut {
@@ -88,7 +95,7 @@ __device__ __forceinline__ int block_exclusive_scan_i32(int v, int* red, int& to
 
 __global__ void __launch_bounds__(kSelThreads)
 select_count_kernel(const float* __restrict__ scores, const float* __restrict__ tau, int Hq, int nb,
-                    int causal, SelCut* __restrict__ cuts) {
+                    int causal, SelCut* __restrict__ cuts, int rule) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int row = blockIdx.x;
   const int bh = row / nb, r = row % nb, h = bh % Hq;
@@ -128,15 +135,25 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
     }
   }
 
-  // fp64 prefix sums over contiguous per-thread segments of the sorted order
   const float t = tau[h];
+  if (rule != kSelThreshold) {
+    // Top-K / ratio: the cut position follows from the candidate count alone
+    if (threadIdx.x == 0) {
+      double kk = rule == kSelTopK ? floor((double)t) : ceil((double)t * (double)n);
+      kk = kk < 1.0 ? 1.0 : (kk > (double)n ? (double)n : kk);   // NaN -> n
+      first_hit = (kk >= 1.0 && kk <= (double)n) ? (int)kk - 1 : n - 1;
+    }
+    __syncthreads();
+  }
+  // fp64 prefix sums over contiguous per-thread segments of the sorted order
+
   const int per = (n + kSelThreads - 1) / kSelThreads;
   const int lo = threadIdx.x * per, hi = min(n, lo + per);
   double seg = 0.0;
   for (int i = lo; i < hi; ++i) seg += (double)key[i];
   double total;
   double run = block_exclusive_scan_f64(seg, red, total);
-  if (t < 1.0f) {
+  if (rule == kSelThreshold && t < 1.0f) {
     for (int i = lo; i < hi; ++i) {
       run += (double)key[i];
       if (run >= (double)t) { atomicMin(&first_hit, i); break; }

@@ -7,7 +7,6 @@
 #include <cuda_runtime.h>
 
 #include "attn_tc.cuh"
-#include "attn_tc2.cuh"
 #include "common.cuh"
 #include "score_tc.cuh"
 #include "select.cuh"
@@ -86,7 +85,8 @@ int check_shape(int B, int Hq, int Hkv, int M, int C, int block) {
 
 template <int C, int G>
 int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
-                    float scale, float* scores, float* part, float* lse_ws, cudaStream_t st) {
+                    int diagonal, float scale, float* scores, float* part, float* lse_ws,
+                    cudaStream_t st) {
   constexpr int BN = 128;
   auto kern = score_tc_kernel<C, G, BN>;
   constexpr int smem = ScoreTc<BN>::kSmem;
@@ -99,21 +99,21 @@ int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
       !make_tile_map(&mk, K, (uint64_t)B * Hkv * rp, S * C, BN))
     return XATTN_ECUDA;
   dim3 grid((rp + 127) / 128, B * Hq);
-  kern<<<grid, kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, scale * kLog2e, part,
-                                            lse_ws, scores);
+  kern<<<grid, kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, diagonal,
+                                            scale * kLog2e, part, lse_ws, scores);
   return launch_status();
 }
 
 template <int C>
 int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
-                   int causal, float scale, float* scores, float* part, float* lse_ws,
-                   cudaStream_t st) {
+                   int causal, int diagonal, float scale, float* scores, float* part,
+                   float* lse_ws, cudaStream_t st) {
   switch (stride) {
-    case 1: return launch_score_tc<C, 128>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 2: return launch_score_tc<C, 64>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 4: return launch_score_tc<C, 32>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 8: return launch_score_tc<C, 16>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
-    case 16: return launch_score_tc<C, 8>(Q, K, B, Hq, Hkv, M, causal, scale, scores, part, lse_ws, st);
+    case 1: return launch_score_tc<C, 128>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
+    case 2: return launch_score_tc<C, 64>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
+    case 4: return launch_score_tc<C, 32>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
+    case 8: return launch_score_tc<C, 16>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
+    case 16: return launch_score_tc<C, 8>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
   }
   return XATTN_EUNSUPPORTED;
 }
@@ -137,25 +137,6 @@ int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* r
   return launch_status();
 }
 
-template <int C, bool DENSE>
-int launch_attn_tc2(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
-                    const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
-                    bf16* O, float* lse, cudaStream_t st) {
-  auto kern = attn_tc2_kernel<C, DENSE>;
-  constexpr int smem = AttnTc2<C>::kSmem;
-  static unsigned long long done = 0;
-  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
-  CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, Q, (uint64_t)B * Hq * M, C) ||
-      !make_tile_map(&mk, K, (uint64_t)B * Hkv * M, C) ||
-      !make_tile_map(&mv, V, (uint64_t)B * Hkv * M, C))
-    return XATTN_ECUDA;
-  dim3 grid(M / 128, B * Hq);
-  kern<<<grid, kAttnTc2Threads, smem, st>>>(mq, mk, mv, row_ptr, col_idx, Hq, Hkv, M, causal,
-                                            scale * kLog2e, O, lse);
-  return launch_status();
-}
-
 template <bool DENSE>
 int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                 const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
@@ -173,19 +154,11 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_
   auto v = static_cast<const bf16*>(V);
   auto o = static_cast<bf16*>(O);
   cudaStream_t st = as_stream(stream);
-#ifndef XATTN_ATTN_SPLIT
   if (C == 64)
     return launch_attn_tc<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                      softmax_scale, o, lse, st);
   return launch_attn_tc<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
                                     softmax_scale, o, lse, st);
-#else
-  if (C == 64)
-    return launch_attn_tc2<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
-                                      softmax_scale, o, lse, st);
-  return launch_attn_tc2<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
-                                     softmax_scale, o, lse, st);
-#endif
 }
 
 }  // namespace
@@ -213,12 +186,14 @@ size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block) {
   return (size_t)B * Hq * rp * (nb + 1) * sizeof(float);
 }
 
-int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C, int stride,
-                int block, int causal, float score_scale, float* scores, void* workspace,
-                size_t workspace_bytes, void* stream) {
+static int score_common(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
+                        int stride, int block, int causal, int pattern, float score_scale,
+                        float* scores, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_shape(B, Hq, Hkv, M, C, block);
   if (rc != XATTN_OK) return rc;
   if (stride <= 0 || block % stride != 0) return XATTN_EINVAL;
+  if (pattern != XATTN_PATTERN_ANTIDIAGONAL && pattern != XATTN_PATTERN_DIAGONAL)
+    return XATTN_EINVAL;
   if (!stride_supported(stride)) return XATTN_EUNSUPPORTED;
   if (B == 0 || Hq == 0 || M == 0) return XATTN_OK;
   if (!Q || !K || !scores || !workspace) return XATTN_EINVAL;
@@ -234,11 +209,26 @@ int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int
   auto q = static_cast<const bf16*>(Q);
   auto k = static_cast<const bf16*>(K);
   cudaStream_t st = as_stream(stream);
+  const int diag = pattern == XATTN_PATTERN_DIAGONAL ? 1 : 0;
   if (C == 64)
-    return launch_score_c<64>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, score_scale, scores,
-                              part, lse_ws, st);
-  return launch_score_c<128>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, score_scale, scores,
-                             part, lse_ws, st);
+    return launch_score_c<64>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, diag, score_scale,
+                              scores, part, lse_ws, st);
+  return launch_score_c<128>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, diag, score_scale,
+                             scores, part, lse_ws, st);
+}
+
+int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C, int stride,
+                int block, int causal, float score_scale, float* scores, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  return score_common(Q, K, B, Hq, Hkv, M, C, stride, block, causal, XATTN_PATTERN_ANTIDIAGONAL,
+                      score_scale, scores, workspace, workspace_bytes, stream);
+}
+
+int xattn_score_ex(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C, int stride,
+                   int block, int causal, int pattern, float score_scale, float* scores,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  return score_common(Q, K, B, Hq, Hkv, M, C, stride, block, causal, pattern, score_scale, scores,
+                      workspace, workspace_bytes, stream);
 }
 
 size_t xattn_select_workspace_size(int B, int Hq, int nb) {
@@ -247,10 +237,11 @@ size_t xattn_select_workspace_size(int B, int Hq, int nb) {
   return (bytes + 255) & ~(size_t)255;
 }
 
-int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
-                 int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
-                 void* workspace, size_t workspace_bytes, void* stream) {
+static int select_common(const float* scores, const float* param, int rule, int B, int Hq, int nb,
+                         int causal, int32_t* row_ptr, int32_t* col_idx, size_t col_capacity,
+                         int32_t* nnz, void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 0 || Hq < 0 || nb < 0) return XATTN_EINVAL;
+  if (rule != kSelThreshold && rule != kSelTopK && rule != kSelRatio) return XATTN_EINVAL;
   const long long rows = (long long)B * Hq * nb;
   if (nb > kSelMaxNb) return XATTN_EUNSUPPORTED;
   // worst-case kept entries must fit the int32 row_ptr
@@ -264,7 +255,7 @@ int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, i
     if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
     return XATTN_OK;
   }
-  if (!scores || !tau || !col_idx || !workspace) return XATTN_EINVAL;
+  if (!scores || !param || !col_idx || !workspace) return XATTN_EINVAL;
   if (workspace_bytes < xattn_select_workspace_size(B, Hq, nb)) return XATTN_EINVAL;
   if (((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
   SelCut* cuts = static_cast<SelCut*>(workspace);
@@ -273,8 +264,8 @@ int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, i
   const int smem = P * 8;
   static unsigned long long done = 0;
   if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
-  select_count_kernel<<<(unsigned)rows, kSelThreads, smem, st>>>(scores, tau, Hq, nb,
-                                                                  causal ? 1 : 0, cuts);
+  select_count_kernel<<<(unsigned)rows, kSelThreads, smem, st>>>(scores, param, Hq, nb,
+                                                                  causal ? 1 : 0, cuts, rule);
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
   const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
   select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
@@ -282,6 +273,20 @@ int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, i
   select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
                                                               row_ptr, col_idx);
   return launch_status();
+}
+
+int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
+                 int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  return select_common(scores, tau, kSelThreshold, B, Hq, nb, causal, row_ptr, col_idx,
+                       col_capacity, nnz, workspace, workspace_bytes, stream);
+}
+
+int xattn_select_ex(const float* scores, const float* param, int rule, int B, int Hq, int nb,
+                    int causal, int32_t* row_ptr, int32_t* col_idx, size_t col_capacity,
+                    int32_t* nnz, void* workspace, size_t workspace_bytes, void* stream) {
+  return select_common(scores, param, rule, B, Hq, nb, causal, row_ptr, col_idx, col_capacity,
+                       nnz, workspace, workspace_bytes, stream);
 }
 
 // ---- selection without a caller workspace -------------------------------
@@ -328,7 +333,8 @@ int xattn_select_noalloc(const float* scores, const float* tau, int B, int Hq, i
   static unsigned long long done = 0;
   if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
   select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, tau, Hq, nb,
-                                                                  causal ? 1 : 0, cuts);
+                                                                  causal ? 1 : 0, cuts,
+                                                                  kSelThreshold);
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
   const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
   select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);

@@ -22,6 +22,8 @@
  *              set reaching a cumulative threshold is taken in descending order.
  *   [DuSA-W3]  DuSA rebuttal, "Response to W3" / "Response to Q1": sparse
  *              attention is then performed within the important blocks only.
+ *   [XA-abl]   XAttention summary, "Measured effects" table: antidiagonal vs
+ *              diagonal scoring; threshold selection vs Top K and fixed Ratio.
  *
  * Conventions shared by every entry point:
  *   - Tensors are device memory owned by the caller, dense and row-major, in the
@@ -105,6 +107,28 @@ XATTN_API int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, 
                 int stride, int block, int causal, float score_scale,
                 float* scores, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Scoring patterns of xattn_score_ex. */
+typedef enum {
+  XATTN_PATTERN_ANTIDIAGONAL = 0,  /* the method: lower-left -> upper-right sums   */
+  XATTN_PATTERN_DIAGONAL = 1       /* the variant the pages compare against        */
+} xattn_pattern;
+
+/*
+ * xattn_score_ex - xattn_score with a choice of pattern [DuSA-Q2, XA-abl].
+ * XATTN_PATTERN_ANTIDIAGONAL is exactly xattn_score. XATTN_PATTERN_DIAGONAL
+ * reads the query rows of each stride group forward, so that X[i',j'] sums the
+ * main diagonal of the S x S tile (i',j') of q k^T instead:
+ *   X[i',j'] = score_scale * sum_s q[i'S+s] . k[j'S+s]
+ * (the diagonal-pattern XAttention variant of DuSA's Response to Q2, and the
+ * "diagonal scoring" row of the XAttention summary's "Measured effects" table,
+ * [XA-abl]). Every other argument, output and error is that of xattn_score;
+ * an unknown pattern returns XATTN_EINVAL.
+ */
+XATTN_API int xattn_score_ex(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
+                             int stride, int block, int causal, int pattern, float score_scale,
+                             float* scores, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
 /*
  * Workspace bytes xattn_select needs: per-row cut (score, index) and count,
  * 12 bytes per (batch, head, query block) row, rounded up to 256 bytes.
@@ -136,6 +160,31 @@ XATTN_API size_t xattn_select_workspace_size(int B, int Hq, int nb);
 XATTN_API int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
                  int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Selection rules of xattn_select_ex. */
+typedef enum {
+  XATTN_SELECT_THRESHOLD = 0,  /* the method: shortest prefix reaching tau[h]     */
+  XATTN_SELECT_TOPK = 1,       /* the floor(param[h]) highest-ranked candidates   */
+  XATTN_SELECT_RATIO = 2       /* ceil(param[h] * candidates) highest-ranked       */
+} xattn_select_rule;
+
+/*
+ * xattn_select_ex - selection with the rules of the ablation [XA-abl].
+ * Candidates are ranked as in xattn_select (score descending, ties to the
+ * smaller block index). param is fp32 [Hq] in device memory:
+ *   XATTN_SELECT_THRESHOLD  param = tau; identical to xattn_select
+ *   XATTN_SELECT_TOPK       keep the first max(1, min(floor(param[h]), n))
+ *   XATTN_SELECT_RATIO      keep the first ceil(param[h] * n), computed in fp64
+ *                           from the fp32 value and clamped to [1, n]
+ * where n is the row's candidate count (r+1 causal, nb otherwise); a NaN param
+ * keeps every candidate. The diagonal block is then added if missing. Outputs,
+ * workspace and capacity behaviour are those of xattn_select; an unknown rule
+ * returns XATTN_EINVAL.
+ */
+XATTN_API int xattn_select_ex(const float* scores, const float* param, int rule, int B, int Hq,
+                              int nb, int causal, int32_t* row_ptr, int32_t* col_idx,
+                              size_t col_capacity, int32_t* nnz, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /*
  * Largest number of selection rows (B*Hq*nb) that xattn_select_noalloc takes.

@@ -50,7 +50,8 @@ import numpy as np
 
 __all__ = [
     "bf16_to_f64", "default_score_scale", "strided_views", "antidiagonal_logits",
-    "block_scores", "select_row", "select_blocks", "selection_margins", "to_csr",
+    "block_scores", "select_row", "select_row_topk", "select_row_ratio", "ratio_count",
+    "select_blocks", "selection_margins", "to_csr",
     "block_sparse_attention", "dense_attention", "layer_block_scores",
     "layer_select", "layer_sparse_attention",
 ]
@@ -175,6 +176,31 @@ def select_row(row: np.ndarray, r: int, tau: float, causal: bool) -> np.ndarray:
     if r not in kept:
         kept.append(r)
     return np.array(sorted(kept), dtype=np.int64)
+
+
+def select_row_topk(row: np.ndarray, r: int, k: int, causal: bool) -> np.ndarray:
+    """Top-K rule of the selection ablation (XAttention summary, "Measured effects"
+    table: threshold selection replaced by Top K): the k highest-scoring candidates
+    (ties to the smaller index), at least one, then the diagonal. Ascending."""
+    nb = row.shape[0]
+    cand = _candidates(r, nb, causal)
+    n = max(1, min(int(k), cand.size))
+    kept = set(int(c) for c in _greedy_order(row, cand)[:n]) | {r}
+    return np.array(sorted(kept), dtype=np.int64)
+
+
+def ratio_count(ratio: float, n: int) -> int:
+    """ceil(ratio * n) taken in fp64 from the given ratio, clamped to [1, n]."""
+    return int(min(n, max(1, np.ceil(np.float64(ratio) * np.float64(n)))))
+
+
+def select_row_ratio(row: np.ndarray, r: int, ratio: float, causal: bool) -> np.ndarray:
+    """Fixed-ratio rule of the selection ablation (XAttention summary, "Measured
+    effects" table: threshold selection replaced by a fixed Ratio): the
+    ceil(ratio * candidates) highest-scoring candidates, then the diagonal."""
+    nb = row.shape[0]
+    cand = _candidates(r, nb, causal)
+    return select_row_topk(row, r, ratio_count(ratio, cand.size), causal)
 
 
 def selection_margins(row: np.ndarray, r: int, tau: float, causal: bool):

@@ -162,3 +162,16 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         xa._load()
     assert "block_sparse_long_04_b200" in sys.modules and importlib  # module itself stays usable
+
+
+def test_unknown_pattern_and_rule_are_rejected():
+    rc = xa._lib.xattn_score_ex(FAKE, FAKE, 1, 4, 2, 1024, 128, 8, 128, 1, 7, 0.03, FAKE, FAKE,
+                                1 << 40, None)
+    assert rc == xa.XATTN_EINVAL
+    rc = xa._lib.xattn_select_ex(FAKE, FAKE, 9, 1, 4, 16, 1, FAKE, FAKE, 1 << 20, FAKE, FAKE,
+                                 1 << 30, None)
+    assert rc == xa.XATTN_EINVAL
+    # the known ones get past these checks and fail later only on the fake stream/device
+    rc = xa._lib.xattn_score_ex(FAKE, FAKE, 1, 4, 2, 1000, 128, 8, 128, 1, 1, 0.03, FAKE, FAKE,
+                                1 << 40, None)
+    assert rc == xa.XATTN_EINVAL   # M not a multiple of the block

@@ -1,0 +1,107 @@
+"""GPU parity of the ablation variants the pages compare against: diagonal-pattern
+scoring, and Top-K / fixed-ratio block selection (XAttention summary, "Measured
+effects" table; DuSA rebuttal, Response to Q2)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from tests import parity as P
+from tests.gpu_util import device_inputs, small_workload
+
+pytestmark = pytest.mark.gpu
+
+xa = pytest.importorskip("block_sparse_long_04_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    yield
+    assert xa.xattn_get_device_error() == xa.XATTN_OK
+
+
+@pytest.mark.parametrize("M,C,Hq,Hkv,S,causal", [
+    (2048, 64, 1, 1, 8, True),
+    (1152, 128, 4, 2, 8, True),
+    (1024, 128, 2, 1, 4, False),
+    (640, 64, 2, 2, 16, True),
+])
+def test_diagonal_pattern_scores(M, C, Hq, Hkv, S, causal):
+    w = small_workload(M, C, Hq, Hkv, S, causal)
+    (Qb, Kb, _), (Q, K, _) = device_inputs(w)
+    nb = M // 128
+    sig = orc.default_score_scale(S, C)
+    scores = torch.empty((1, Hq, nb, nb), device="cuda")
+    ws = torch.empty(xa.xattn_score_workspace_size(1, Hq, M, S), dtype=torch.uint8, device="cuda")
+    xa.xattn_score_ex(Q, K, S, causal, xa.XATTN_PATTERN_DIAGONAL, sig, scores, ws)
+    diag = scores.cpu().numpy()
+    ref = orc.layer_block_scores(Qb, Kb, Hkv, S, 128, sig, causal, antidiagonal=False)
+    for h in range(Hq):
+        P.assert_scores_close(diag[0, h], ref[(0, h)], f"diagonal scores head {h}")
+    # and the antidiagonal pattern through the same entry point is xattn_score
+    anti = torch.empty_like(scores)
+    xa.xattn_score_ex(Q, K, S, causal, xa.XATTN_PATTERN_ANTIDIAGONAL, sig, anti, ws)
+    base = torch.empty_like(scores)
+    xa.xattn_score(Q, K, S, causal, sig, base, ws)
+    assert torch.equal(anti, base)
+    if M >= 1024:
+        assert not torch.allclose(anti, scores)
+
+
+def _select_ex(scores_np, param, rule, causal):
+    B, Hq, nb, _ = scores_np.shape
+    sc = torch.from_numpy(np.ascontiguousarray(scores_np, dtype=np.float32)).cuda()
+    pr = torch.tensor(param, dtype=torch.float32, device="cuda")
+    row_ptr = torch.empty(B * Hq * nb + 1, dtype=torch.int32, device="cuda")
+    col = torch.empty(xa.max_kept(B, Hq, nb, causal), dtype=torch.int32, device="cuda")
+    nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8, device="cuda")
+    xa.xattn_select_ex(sc, pr, rule, causal, row_ptr, col, nnz, ws)
+    return row_ptr.cpu().numpy(), col.cpu().numpy(), int(nnz.item())
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("nb", [1, 5, 64, 333])
+def test_topk_and_ratio_selection_exact(causal, nb):
+    """Top-K and ratio depend on the ranking only: bit-exact against the oracle
+    given the same fp32 scores (ties included)."""
+    rng = np.random.default_rng(nb * 3 + causal)
+    Hq = 3
+    s = rng.gamma(0.3, size=(1, Hq, nb, nb))
+    s[0, 2] = np.round(s[0, 2] * 4) / 4          # head 2: many exact ties
+    if causal:
+        s = np.tril(s)
+    s = (s / np.maximum(s.sum(-1, keepdims=True), 1e-30)).astype(np.float32)
+    s64 = s.astype(np.float64)
+    for rule, param, fn in ((xa.XATTN_SELECT_TOPK, [1.0, 7.5, 3.0], orc.select_row_topk),
+                            (xa.XATTN_SELECT_RATIO, [0.1, 0.33, 1.0], orc.select_row_ratio)):
+        rp, col, nnz = _select_ex(s, param, rule, causal)
+        assert nnz == rp[-1]
+        for h in range(Hq):
+            p = np.float32(param[h])
+            for r in range(nb):
+                want = fn(s64[0, h, r], r, int(np.floor(p)) if rule == xa.XATTN_SELECT_TOPK
+                          else float(p), causal)
+                got = col[rp[h * nb + r]:rp[h * nb + r + 1]]
+                np.testing.assert_array_equal(got, want, err_msg=f"rule {rule} h{h} r{r}")
+
+
+def test_threshold_rule_equals_select():
+    rng = np.random.default_rng(1)
+    nb, Hq = 200, 2
+    s = np.tril(rng.gamma(0.3, size=(1, Hq, nb, nb)))
+    s = (s / s.sum(-1, keepdims=True)).astype(np.float32)
+    a = _select_ex(s, [0.9, 0.6], xa.XATTN_SELECT_THRESHOLD, True)
+    sc = torch.from_numpy(s).cuda()
+    tau = torch.tensor([0.9, 0.6], device="cuda")
+    row_ptr = torch.empty(Hq * nb + 1, dtype=torch.int32, device="cuda")
+    col = torch.empty(xa.max_kept(1, Hq, nb, True), dtype=torch.int32, device="cuda")
+    nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(xa.xattn_select_workspace_size(1, Hq, nb), dtype=torch.uint8, device="cuda")
+    xa.xattn_select(sc, tau, True, row_ptr, col, nnz, ws)
+    n = int(nnz.item())
+    assert a[2] == n
+    np.testing.assert_array_equal(a[0], row_ptr.cpu().numpy())
+    np.testing.assert_array_equal(a[1][:n], col.cpu().numpy()[:n])

@@ -226,6 +226,45 @@ def test_selection_special_cases():
     assert orc.select_row(exact, 0, 0.75, False).tolist() == [0, 1]
 
 
+@pytest.mark.parametrize("seed", range(30))
+def test_topk_and_ratio_keep_the_heaviest_k(seed):
+    """Brute force over all k-subsets: the Top-K set has the largest mass among
+    sets of its size, and the ratio rule keeps ceil(ratio * candidates)."""
+    rng = np.random.default_rng(100 + seed)
+    nb = int(rng.integers(2, 10))
+    causal = bool(seed % 2)
+    r = int(rng.integers(0, nb))
+    row = rng.gamma(0.5, size=nb)
+    if causal:
+        row[r + 1:] = 0.0
+    row /= row.sum()
+    cand = list(range(r + 1)) if causal else list(range(nb))
+    k = int(rng.integers(1, len(cand) + 2))
+    kept = set(orc.select_row_topk(row, r, k, causal).tolist())
+    n = min(k, len(cand))
+    T = kept if len(kept) == n else kept - {r}
+    assert len(T) == n and T <= set(cand) and r in kept
+    best = max(sum(row[list(H)]) for H in itertools.combinations(cand, n))
+    assert math.isclose(sum(row[list(T)]), best, rel_tol=1e-12)
+    ratio = float(rng.uniform(0.01, 1.0))
+    kr = set(orc.select_row_ratio(row, r, ratio, causal).tolist())
+    nr = math.ceil(ratio * len(cand))
+    assert len(kr - {r}) in (nr, nr - 1) and len(kr) in (nr, nr + 1)
+
+
+def test_topk_ratio_special_cases():
+    row = np.array([0.1, 0.4, 0.2, 0.3])
+    assert orc.select_row_topk(row, 0, 1, False).tolist() == [0, 1]
+    assert orc.select_row_topk(row, 3, 2, False).tolist() == [1, 3]
+    assert orc.select_row_topk(row, 3, 99, False).tolist() == [0, 1, 2, 3]
+    assert orc.select_row_topk(row, 2, 0, True).tolist() == [1, 2]      # at least one
+    assert orc.select_row_ratio(row, 0, 0.5, False).tolist() == [0, 1, 3]
+    assert orc.select_row_ratio(row, 0, 1.0, False).tolist() == [0, 1, 2, 3]
+    assert orc.ratio_count(1e-9, 5) == 1 and orc.ratio_count(0.2, 10) == 2
+    tie = np.array([0.25, 0.25, 0.25, 0.25])
+    assert orc.select_row_topk(tie, 3, 2, False).tolist() == [0, 1, 3]
+
+
 def test_margins_agree_with_selection():
     rng = np.random.default_rng(3)
     for _ in range(50):
