@@ -5,18 +5,24 @@
 // block r) tile of 128 query rows; GQA maps query head h to KV head h/(Hq/Hkv).
 //
 // Warp roles (256 threads):
-//   warp 0, one lane  TMA producer: Q once, then K/V tiles of the kept blocks
-//                     (in list order) into a ring of kStages shared-memory stages.
+//   warp 0, one lane  TMA producer: Q once, then the K and V tiles of the kept
+//                     blocks (in list order) into two rings of kStages stages with
+//                     their own full/empty barriers; K runs one block ahead of V.
 //   warp 1, one lane  MMA issuer: S = Q K^T into TMEM (128 lanes x 128 fp32 cols),
 //                     then O += P V into TMEM (128 lanes x C fp32 cols). S of block
 //                     j+1 is issued as soon as the softmax has read S of block j, so
 //                     it overlaps that softmax.
-//   warps 4-7         softmax, one query row per thread (TMEM lane = row): read the
-//                     S row, causal mask on the diagonal block, online softmax in
-//                     fp32 (base 2) with lazy rescaling (O and l are rescaled only
-//                     when the running max grows by more than 2^8), write P as bf16
-//                     into shared memory in the tensor core's 128-byte-swizzled
-//                     K-major layout, and finally normalise O out of TMEM.
+//   warps 4-11        softmax, two threads per query row (TMEM lane = row): warps
+//                     4-7 take keys 0-63 of each block, warps 8-11 keys 64-127, so
+//                     every sub-partition runs two softmax warps whose
+//                     exponentials interleave. Per block: read the half row of S,
+//                     causal mask on the diagonal block, half-row max exchanged
+//                     through shared memory (an mbarrier per block), online
+//                     softmax in fp32 (base 2) with lazy rescaling (O and l are
+//                     rescaled only when the running max grows by more than 2^8),
+//                     P as bf16 into shared memory in the tensor core's
+//                     128-byte-swizzled K-major layout; finally each half
+//                     normalises its half of the O columns out of TMEM.
 // Every wait is bounded (sm100::mbar_wait); on a timeout the CTA raises
 // XATTN_ETIMEOUT, every role stops, in-flight copies and MMAs are drained, and
 // TMEM is freed before the CTA exits.
@@ -26,7 +32,7 @@
 
 namespace xattn {
 
-constexpr int kAttnTcThreads = 256;
+constexpr int kAttnTcThreads = 384;
 
 template <int C>
 struct AttnTc {
@@ -39,7 +45,8 @@ struct AttnTc {
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffP = kOffV + kStages * kTile;   // 128 x 128 bf16
   static constexpr int kOffBar = kOffP + 2 * kRegion;
-  static constexpr int kSmem = kOffBar + 256 + 1024;      // + alignment slack
+  static constexpr int kOffX = kOffBar + 256;             // half-row max / sum exchange
+  static constexpr int kSmem = kOffX + 6 * 128 * 4 + 1024;  // + alignment slack
   static constexpr int kTmemCols = 256;                   // S: 0..127, O: 128..128+C-1
 };
 
@@ -60,15 +67,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t sV0 = smem_u32(smem + L::kOffV);
   const uint32_t sP = smem_u32(smem + L::kOffP);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + ST;
-  uint64_t* q_full = bars + 2 * ST;
+  uint64_t* k_full = bars;            // [ST] K tile of a block landed
+  uint64_t* k_empty = bars + ST;      // [ST] its S MMA completed
+  uint64_t* v_full = bars + 2 * ST;   // [ST] V tile of a block landed
+  uint64_t* v_empty = bars + 3 * ST;  // [ST] its PV MMA completed
+  uint64_t* q_full = bars + 4 * ST;
   uint64_t* s_full = q_full + 1;
   uint64_t* s_free = q_full + 2;
   uint64_t* p_full = q_full + 3;
   uint64_t* o_done = q_full + 4;
   uint64_t* drain = q_full + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 6);
+  uint64_t* x_full = q_full + 6;    // [2] half-row maxima of a block published
+  uint64_t* l_full = q_full + 8;    // half-row sums published (epilogue)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 9);
+  float* xmax = reinterpret_cast<float*>(smem + L::kOffX);   // [2 parity][2 half][128]
+  float* xsum = xmax + 4 * 128;                              // [2 half][128]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -86,13 +99,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   };
 
   if (tid == 0) {
-    for (int i = 0; i < ST; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+    }
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
+    mbar_init(s_free, 8);
+    mbar_init(p_full, 8);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
+    mbar_init(&x_full[0], 8);
+    mbar_init(&x_full[1], 8);
+    mbar_init(l_full, 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -119,25 +138,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int g = 0; g < L::kNReg; ++g) tma_load_2d(sQ + g * L::kRegion, &tmQ, g * 64, yq, q_full);
       const int ykv = (b * Hkv + kvh) * M;
-      int j = 0;
+      // K of block j is issued before V of block j-1: S of a block needs only its
+      // K tile, so K loads run one block ahead and are never queued behind the
+      // wait for an older PV to free a V stage
+      auto load_v = [&](int jv, int cv) -> bool {
+        const int st = jv % ST;
+        if (jv >= ST && !mbar_wait(&v_empty[st], ((jv / ST) - 1) & 1, abort_flag)) return false;
+        mbar_expect_tx(&v_full[st], L::kTile);
+#pragma unroll
+        for (int g = 0; g < L::kNReg; ++g)
+          tma_load_2d(sV0 + st * L::kTile + g * L::kRegion, &tmV, g * 64, ykv + cv * 128, &v_full[st]);
+        return true;
+      };
+      int nk = 0, nv = 0, c_prev = -1;
+      bool ok = true;
       for (int it = beg; it < end; ++it) {
         const int c = block_of(it);
         if (c < 0) continue;
-        const int st = j % ST;
-        if (j >= ST && !mbar_wait(&kv_empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(&kv_full[st], 2 * L::kTile);
+        const int st = nk % ST;
+        if (nk >= ST && !(ok = mbar_wait(&k_empty[st], ((nk / ST) - 1) & 1, abort_flag))) break;
+        mbar_expect_tx(&k_full[st], L::kTile);
 #pragma unroll
-        for (int g = 0; g < L::kNReg; ++g) {
-          tma_load_2d(sK0 + st * L::kTile + g * L::kRegion, &tmK, g * 64, ykv + c * 128, &kv_full[st]);
-          tma_load_2d(sV0 + st * L::kTile + g * L::kRegion, &tmV, g * 64, ykv + c * 128, &kv_full[st]);
+        for (int g = 0; g < L::kNReg; ++g)
+          tma_load_2d(sK0 + st * L::kTile + g * L::kRegion, &tmK, g * 64, ykv + c * 128, &k_full[st]);
+        ++nk;
+        if (c_prev >= 0) {
+          if (!(ok = load_v(nv, c_prev))) break;
+          ++nv;
         }
-        ++j;
+        c_prev = c;
       }
+      if (ok && c_prev >= 0 && load_v(nv, c_prev)) ++nv;
       // drain: every load issued must land before the CTA may exit
       volatile int no_abort = 0;
       mbar_wait(q_full, 0, &no_abort);
-      for (int jj = (j > ST ? j - ST : 0); jj < j; ++jj)
-        mbar_wait(&kv_full[jj % ST], (jj / ST) & 1, &no_abort);
+      for (int jj = (nk > ST ? nk - ST : 0); jj < nk; ++jj)
+        mbar_wait(&k_full[jj % ST], (jj / ST) & 1, &no_abort);
+      for (int jj = (nv > ST ? nv - ST : 0); jj < nv; ++jj)
+        mbar_wait(&v_full[jj % ST], (jj / ST) & 1, &no_abort);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -155,24 +193,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                      smem_desc_sw128(sK0 + st * L::kTile + off, 16, 1024), idS, kk > 0);
         }
         mma_commit(s_full);
+        mma_commit(&k_empty[st]);
       };
       bool ok = n > 0 && mbar_wait(q_full, 0, abort_flag);
-      if (ok) ok = mbar_wait(&kv_full[0], 0, abort_flag);
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_S(0);
       }
       for (int j = 0; ok && j < n; ++j) {
         if (j + 1 < n) {
-          ok = mbar_wait(&kv_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag) &&
+          ok = mbar_wait(&k_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag) &&
                mbar_wait(s_free, j & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_S(j + 1);
         }
-        if (!(ok = mbar_wait(p_full, j & 1, abort_flag))) break;
-        tc_fence_after();
         const int st = j % ST;
+        ok = mbar_wait(p_full, j & 1, abort_flag) && mbar_wait(&v_full[st], (j / ST) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t a_off = (kk >> 2) * L::kRegion + (kk & 3) * 32;
@@ -181,7 +221,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                      (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(o_done);
-        mma_commit(&kv_empty[st]);
+        mma_commit(&v_empty[st]);
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       mma_commit(drain);
@@ -190,40 +230,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
+    const int half = (warp >= 8) ? 1 : 0;              // keys [64*half, 64*half + 64)
     const int q_row = (warp & 3) * 32 + lane;          // row within the query block
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    float m = kNegInf, l = 0.f;
+    const int k0 = half * 64;
+    float m = kNegInf, l = 0.f;                        // l: this half's share of the sum
     int j = 0;
     bool ok = true;
-    float s[128];
     for (int it = beg; it < end; ++it) {
       const int c = block_of(it);
       if (c < 0) continue;
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + lane_off + q * 32, s + q * 32);
+      float s[64];
+      tmem_ld32(tS + lane_off + k0, s);
+      tmem_ld32(tS + lane_off + k0 + 32, s + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
 
-      // row max of the raw logits (the scale is positive); masked keys of the
-      // diagonal block are set to -inf first, on the diagonal block only
+      // half-row max of the raw logits (the scale is positive); masked keys of
+      // the diagonal block are set to -inf first, on the diagonal block only
       if (causal && c == r) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = (i > q_row) ? kNegInf : s[i];
+        for (int i = 0; i < 64; ++i) s[i] = (k0 + i > q_row) ? kNegInf : s[i];
       }
       // eight independent partial maxima / sums keep the reductions off one
-      // 128-long dependency chain
+      // long dependency chain
       float pm[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) pm[k] = s[k];
 #pragma unroll
-      for (int i = 8; i < 128; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+      for (int i = 8; i < 64; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
+      const float hm = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                              fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      // exchange with the other half of the row (double-buffered by block parity)
+      float* xm = xmax + (j & 1) * 256;
+      xm[half * 128 + q_row] = hm;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&x_full[j & 1]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&x_full[j & 1], (j >> 1) & 1, abort_flag));
+      if (!ok) break;
+      const float mx = fmaxf(hm, xm[(half ^ 1) * 128 + q_row]);
+
       const float m_new = fmaxf(m, mx * scale_log2);
       float corr = 1.f;
       bool resc = false;
@@ -237,7 +288,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float neg_m = -m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < 64; ++i) {
         s[i] = ex2(fmaf(s[i], scale_log2, neg_m));
         ps[i & 7] += s[i];
       }
@@ -251,26 +302,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, resc)) {
+        // this half rescales its half of the O columns
 #pragma unroll
-        for (int q = 0; q < C / 32; ++q) {
+        for (int q = 0; q < C / 64; ++q) {
           float o[32];
-          tmem_ld32(tO + lane_off + q * 32, o);
+          const uint32_t ta = tO + lane_off + half * (C / 2) + q * 32;
+          tmem_ld32(ta, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= corr;
-          tmem_st32(tO + lane_off + q * 32, o);
+          tmem_st32(ta, o);
         }
         tmem_wait_st();
       }
-      // P row -> shared memory, 128-byte swizzled K-major (two 64-key regions)
+      // P half row -> shared memory region `half`, 128-byte swizzled K-major
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
+      for (int ch = 0; ch < 8; ++ch) {
         uint4 v;
         v.x = pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]);
         v.y = pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]);
         v.z = pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]);
         v.w = pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]);
-        const uint32_t addr = sP + (ch >> 3) * L::kRegion + q_row * 128 + (((ch & 7) ^ (q_row & 7)) << 4);
+        const uint32_t addr = sP + half * L::kRegion + q_row * 128 + ((ch ^ (q_row & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                      "r"(v.z), "r"(v.w) : "memory");
       }
@@ -281,17 +334,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ++j;
     }
 
-    // epilogue: O / l -> bf16 global; lse = (m + log2 l) ln 2
-    bf16* orow = O + ((size_t)bh * M + (size_t)r * 128 + q_row) * C;
+    // epilogue: the row sum is the two halves' shares; each half normalises and
+    // writes its half of the O columns; lse = (m + log2 l) ln 2
+    if (ok) {
+      xsum[half * 128 + q_row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_full);
+      ok = __all_sync(0xffffffffu, mbar_wait(l_full, 0, abort_flag));
+    }
+    const float lt = ok ? xsum[q_row] + xsum[128 + q_row] : 0.f;
+    bf16* orow = O + ((size_t)bh * M + (size_t)r * 128 + q_row) * C + half * (C / 2);
     if (ok && j > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll
-        for (int q = 0; q < C / 32; ++q) {
+        for (int q = 0; q < C / 64; ++q) {
           float o[32];
-          tmem_ld32(tO + lane_off + q * 32, o);
+          tmem_ld32(tO + lane_off + half * (C / 2) + q * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
@@ -303,14 +364,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
           }
         }
-        if (lse != nullptr)
-          lse[(size_t)bh * M + (size_t)r * 128 + q_row] = l > 0.f ? (m + lg2(l)) * kLn2 : kNegInf;
+        if (lse != nullptr && half == 0)
+          lse[(size_t)bh * M + (size_t)r * 128 + q_row] = lt > 0.f ? (m + lg2(lt)) * kLn2 : kNegInf;
       }
     } else if (ok && j == 0) {
       const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int i = 0; i < C; i += 8) *reinterpret_cast<uint4*>(orow + i) = z;
-      if (lse != nullptr) lse[(size_t)bh * M + (size_t)r * 128 + q_row] = kNegInf;
+      for (int i = 0; i < C / 2; i += 8) *reinterpret_cast<uint4*>(orow + i) = z;
+      if (lse != nullptr && half == 0) lse[(size_t)bh * M + (size_t)r * 128 + q_row] = kNegInf;
     }
     tc_fence_before();
   }

@@ -87,7 +87,10 @@ template <int C, int G>
 int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
                     int diagonal, float scale, float* scores, float* part, float* lse_ws,
                     cudaStream_t st) {
-  constexpr int BN = 128;
+#ifndef XATTN_SCORE_BN
+#define XATTN_SCORE_BN 128
+#endif
+  constexpr int BN = XATTN_SCORE_BN;
   auto kern = score_tc_kernel<C, G, BN>;
   constexpr int smem = ScoreTc<BN>::kSmem;
   static unsigned long long done = 0;
