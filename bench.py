@@ -185,6 +185,23 @@ def config_of(w):
             "parallelism": "one independent layer per GPU (no collective)"}
 
 
+# ------------------------------------------------------- multi-rank helpers
+def dist_max(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (the job time is the slowest rank)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(total_ms_max: float, steps: int, world: int, batch: int) -> float:
+    """Whole-job ms per layer: every rank processed `steps` layers of `batch`
+    sequences in `total_ms_max` (max over ranks) milliseconds."""
+    return total_ms_max / (steps * world * batch)
+
+
 # ------------------------------------------------------------ our arm
 def main():
     a = parse()
@@ -211,11 +228,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(x, dist, dev)
 
     # inputs: generated on the host (pinned), copied once; resident in HBM when timed
     seed = a.seed + rank
@@ -267,7 +280,7 @@ def main():
     barrier()
     total_ms = max_over_ranks(t0.elapsed_time(t1))
     ms_step = total_ms / a.steps
-    value = total_ms / (a.steps * world * w.B)        # ms per layer, whole job
+    value = job_ms_per_layer(total_ms, a.steps, world, w.B)   # ms per layer, whole job
     st_score = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     st_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     st_attn = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -345,7 +358,7 @@ def main():
         e2e_total = max_over_ranks(e0.elapsed_time(e1))
         h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh)) + tau_np.nbytes
         d2h = Oh.numel() * Oh.element_size()
-        e2e = {"value": e2e_total / (a.steps * world * w.B), "unit": UNIT,
+        e2e = {"value": job_ms_per_layer(e2e_total, a.steps, world, w.B), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del Oh
 

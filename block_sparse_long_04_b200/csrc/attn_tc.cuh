@@ -4,25 +4,29 @@
 // W3/Q1; XAttention summary, Approach). One CTA = one (batch, query head, query
 // block r) tile of 128 query rows; GQA maps query head h to KV head h/(Hq/Hkv).
 //
-// Warp roles (256 threads):
+// Warp roles (384 threads):
 //   warp 0, one lane  TMA producer: Q once, then the K and V tiles of the kept
 //                     blocks (in list order) into two rings of kStages stages with
 //                     their own full/empty barriers; K runs one block ahead of V.
-//   warp 1, one lane  MMA issuer: S = Q K^T into TMEM (128 lanes x 128 fp32 cols),
-//                     then O += P V into TMEM (128 lanes x C fp32 cols). S of block
-//                     j+1 is issued as soon as the softmax has read S of block j, so
-//                     it overlaps that softmax.
+//   warp 1, one lane  MMA issuer and TMEM owner: S = Q K^T into TMEM (128 lanes x
+//                     128 fp32 columns); S of block j+1 is issued as soon as the
+//                     softmax has read S of block j. Then, per key half g (keys
+//                     64g..64g+63), O_g += P_g V_g into its own TMEM accumulator.
 //   warps 4-11        softmax, two threads per query row (TMEM lane = row): warps
-//                     4-7 take keys 0-63 of each block, warps 8-11 keys 64-127, so
-//                     every sub-partition runs two softmax warps whose
-//                     exponentials interleave. Per block: read the half row of S,
-//                     causal mask on the diagonal block, half-row max exchanged
-//                     through shared memory (an mbarrier per block), online
-//                     softmax in fp32 (base 2) with lazy rescaling (O and l are
-//                     rescaled only when the running max grows by more than 2^8),
-//                     P as bf16 into shared memory in the tensor core's
-//                     128-byte-swizzled K-major layout; finally each half
-//                     normalises its half of the O columns out of TMEM.
+//                     4-7 own keys 0-63 of every block, warps 8-11 keys 64-127.
+//                     The two halves are independent online softmaxes over
+//                     disjoint key sets (own running max m_g, sum l_g, accumulator
+//                     O_g), so they never wait for each other inside the loop; at
+//                     the end they are merged exactly:
+//                       m = max(m_0, m_1), l = sum_g l_g 2^(m_g - m),
+//                       O = sum_g O_g 2^(m_g - m) / l.
+//                     Per block: read the half row of S, causal mask on the
+//                     diagonal block, fp32 base-2 softmax with the scale folded into
+//                     one FMA, lazy rescaling (O_g and l_g are rescaled only when
+//                     m_g grows by more than 2^8), P_g as bf16 into shared memory in
+//                     the tensor core's 128-byte-swizzled K-major layout.
+// Every role walks the row's list with the next entry's load already in flight
+// (ListIter), so no role waits on a global load inside its loop.
 // Every wait is bounded (sm100::mbar_wait); on a timeout the CTA raises
 // XATTN_ETIMEOUT, every role stops, in-flight copies and MMAs are drained, and
 // TMEM is freed before the CTA exits.
@@ -43,11 +47,41 @@ struct AttnTc {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffP = kOffV + kStages * kTile;   // 128 x 128 bf16
+  static constexpr int kOffP = kOffV + kStages * kTile;   // 128 x 128 bf16, region g = half g
   static constexpr int kOffBar = kOffP + 2 * kRegion;
-  static constexpr int kOffX = kOffBar + 256;             // half-row max / sum exchange
-  static constexpr int kSmem = kOffX + 6 * 128 * 4 + 1024;  // + alignment slack
-  static constexpr int kTmemCols = 256;                   // S: 0..127, O: 128..128+C-1
+  static constexpr int kOffX = kOffBar + 256;             // end-of-row (m, l) exchange
+  static constexpr int kSmem = kOffX + 2 * 128 * 8 + 1024;  // + alignment slack
+  static constexpr int kTmemCols = 512;                   // S 0..127, O_0 128.., O_1 256..
+  static constexpr int kColS = 0;
+  static constexpr int kColO = 128;                       // + g * 128
+};
+
+// Walks the kept-block list of one row, skipping entries outside [0, nb) and,
+// when causal, above the diagonal; the load of the following entry is issued as
+// soon as the current one is returned, so its latency overlaps the caller's work.
+struct ListIter {
+  const int32_t* col;
+  int it, end, nb, r;
+  bool causal, dense;
+  int raw;
+  __device__ __forceinline__ int fetch(int i) const {
+    return i < end ? (dense ? i : __ldg(col + i)) : -1;
+  }
+  __device__ __forceinline__ void init(const int32_t* c, int beg, int e, int nb_, int r_,
+                                       bool causal_, bool dense_) {
+    col = c; it = beg; end = e; nb = nb_; r = r_; causal = causal_; dense = dense_;
+    raw = fetch(it);
+  }
+  // next valid key block, or -1 at the end of the list
+  __device__ __forceinline__ int next() {
+    while (it < end) {
+      const int c = raw;
+      ++it;
+      raw = fetch(it);
+      if (c >= 0 && c < nb && !(causal && c > r)) return c;
+    }
+    return -1;
+  }
 };
 
 template <int C, bool DENSE>
@@ -70,19 +104,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* k_full = bars;            // [ST] K tile of a block landed
   uint64_t* k_empty = bars + ST;      // [ST] its S MMA completed
   uint64_t* v_full = bars + 2 * ST;   // [ST] V tile of a block landed
-  uint64_t* v_empty = bars + 3 * ST;  // [ST] its PV MMA completed
+  uint64_t* v_empty = bars + 3 * ST;  // [ST] both of its PV MMAs completed
   uint64_t* q_full = bars + 4 * ST;
-  uint64_t* s_full = q_full + 1;
-  uint64_t* s_free = q_full + 2;
-  uint64_t* p_full = q_full + 3;
-  uint64_t* o_done = q_full + 4;
-  uint64_t* drain = q_full + 5;
-  uint64_t* x_full = q_full + 6;    // [2] half-row maxima of a block published
-  uint64_t* l_full = q_full + 8;    // half-row sums published (epilogue)
+  uint64_t* s_full = q_full + 1;      // S of the current block computed
+  uint64_t* s_free = q_full + 2;      // all 8 softmax warps have read it
+  uint64_t* p_full = q_full + 3;      // [2] P_g written (4 warps each)
+  uint64_t* o_done = q_full + 5;      // [2] PV_g of the block completed
+  uint64_t* drain = q_full + 7;
+  uint64_t* x_full = q_full + 8;      // end-of-row (m_g, l_g) published (8 warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 9);
-  float* xmax = reinterpret_cast<float*>(smem + L::kOffX);   // [2 parity][2 half][128]
-  float* xsum = xmax + 4 * 128;                              // [2 half][128]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* xchg = reinterpret_cast<float2*>(smem + L::kOffX);   // [2 half][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = M / 128;
@@ -93,10 +125,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   int beg, end;
   if (DENSE) { beg = 0; end = causal ? r + 1 : nb; }
   else { beg = row_ptr[row]; end = row_ptr[row + 1]; }
-  auto block_of = [&](int it) -> int {
-    const int c = DENSE ? it : __ldg(col_idx + it);
-    return (c < 0 || c >= nb || (causal && c > r)) ? -1 : c;
-  };
 
   if (tid == 0) {
     for (int i = 0; i < ST; ++i) {
@@ -106,12 +134,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);
-    mbar_init(p_full, 8);
-    mbar_init(o_done, 1);
+    mbar_init(&p_full[0], 4); mbar_init(&p_full[1], 4);
+    mbar_init(&o_done[0], 1); mbar_init(&o_done[1], 1);
     mbar_init(drain, 1);
-    mbar_init(&x_full[0], 8);
-    mbar_init(&x_full[1], 8);
-    mbar_init(l_full, 8);
+    mbar_init(x_full, 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -128,7 +154,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tS = tmem + L::kColS;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -150,11 +176,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tma_load_2d(sV0 + st * L::kTile + g * L::kRegion, &tmV, g * 64, ykv + cv * 128, &v_full[st]);
         return true;
       };
+      ListIter li;
+      li.init(col_idx, beg, end, nb, r, causal != 0, DENSE);
       int nk = 0, nv = 0, c_prev = -1;
       bool ok = true;
-      for (int it = beg; it < end; ++it) {
-        const int c = block_of(it);
-        if (c < 0) continue;
+      for (int c = li.next(); c >= 0; c = li.next()) {
         const int st = nk % ST;
         if (nk >= ST && !(ok = mbar_wait(&k_empty[st], ((nk / ST) - 1) & 1, abort_flag))) break;
         mbar_expect_tx(&k_full[st], L::kTile);
@@ -180,8 +206,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      int n = 0;
-      for (int it = beg; it < end; ++it) n += block_of(it) >= 0 ? 1 : 0;
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, C, false, true);
       auto issue_S = [&](int j) {
@@ -195,33 +219,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(s_full);
         mma_commit(&k_empty[st]);
       };
-      bool ok = n > 0 && mbar_wait(q_full, 0, abort_flag);
+      ListIter li;
+      li.init(col_idx, beg, end, nb, r, causal != 0, DENSE);
+      bool have_cur = li.next() >= 0;
+      bool have_nxt = have_cur && li.next() >= 0;
+      bool ok = have_cur && mbar_wait(q_full, 0, abort_flag);
       if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_S(0);
       }
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n) {
+      for (int j = 0; ok && have_cur; ++j) {
+        const int st = j % ST;
+        if (have_nxt) {
           ok = mbar_wait(&k_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag) &&
                mbar_wait(s_free, j & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_S(j + 1);
         }
-        const int st = j % ST;
-        ok = mbar_wait(p_full, j & 1, abort_flag) && mbar_wait(&v_full[st], (j / ST) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
+        if (!(ok = mbar_wait(&v_full[st], (j / ST) & 1, abort_flag))) break;
+        for (int g = 0; g < 2; ++g) {
+          if (!(ok = mbar_wait(&p_full[g], j & 1, abort_flag))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a_off = (kk >> 2) * L::kRegion + (kk & 3) * 32;
-          mma_f16_ss(tO, smem_desc_sw128(sP + a_off, 16, 1024),
-                     smem_desc_sw128(sV0 + st * L::kTile + kk * 2048, L::kRegion, 1024), idPV,
-                     (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {   // keys 64g + 16kk .. +15
+            mma_f16_ss(tmem + L::kColO + g * 128,
+                       smem_desc_sw128(sP + g * L::kRegion + kk * 32, 16, 1024),
+                       smem_desc_sw128(sV0 + st * L::kTile + (g * 4 + kk) * 2048, L::kRegion, 1024),
+                       idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&o_done[g]);
         }
-        mma_commit(o_done);
+        if (!ok) break;
         mma_commit(&v_empty[st]);
+        have_cur = have_nxt;
+        have_nxt = have_cur && li.next() >= 0;
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
       mma_commit(drain);
@@ -230,22 +263,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
-    const int half = (warp >= 8) ? 1 : 0;              // keys [64*half, 64*half + 64)
+    const int g = (warp >= 8) ? 1 : 0;                 // keys [64g, 64g + 64) of each block
     const int q_row = (warp & 3) * 32 + lane;          // row within the query block
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const int k0 = half * 64;
-    float m = kNegInf, l = 0.f;                        // l: this half's share of the sum
+    const uint32_t tSg = tS + lane_off + g * 64;
+    const uint32_t tOg = tmem + lane_off + L::kColO + g * 128;
+    const int k0 = g * 64;
+    float m = kNegInf, l = 0.f;
     int j = 0;
     bool ok = true;
-    for (int it = beg; it < end; ++it) {
-      const int c = block_of(it);
-      if (c < 0) continue;
+    ListIter li;
+    li.init(col_idx, beg, end, nb, r, causal != 0, DENSE);
+    for (int c = li.next(); c >= 0; c = li.next()) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float s[64];
-      tmem_ld32(tS + lane_off + k0, s);
-      tmem_ld32(tS + lane_off + k0 + 32, s + 32);
+      tmem_ld32(tSg, s);
+      tmem_ld32(tSg + 32, s + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -264,28 +299,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int k = 0; k < 8; ++k) pm[k] = s[k];
 #pragma unroll
       for (int i = 8; i < 64; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
-      const float hm = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                              fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      // exchange with the other half of the row (double-buffered by block parity)
-      float* xm = xmax + (j & 1) * 256;
-      xm[half * 128 + q_row] = hm;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&x_full[j & 1]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&x_full[j & 1], (j >> 1) & 1, abort_flag));
-      if (!ok) break;
-      const float mx = fmaxf(hm, xm[(half ^ 1) * 128 + q_row]);
-
+      // a row may see no key of this half (the upper half of the diagonal block)
       const float m_new = fmaxf(m, mx * scale_log2);
       float corr = 1.f;
       bool resc = false;
-      if (j == 0) {
+      if (m == kNegInf) {
         m = m_new;
       } else if (m_new > m + 8.f) {
         corr = ex2(m - m_new);
         m = m_new;
         resc = true;
       }
-      const float neg_m = -m;
+      const float neg_m = (m == kNegInf) ? 0.f : -m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
@@ -295,27 +322,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l = l * corr + rs;
 
-      // PV of the previous block must be complete: P buffer free, O stable
+      // PV_g of the previous block must be complete: P_g free, O_g stable
       if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[g], (j - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
       }
       if (__any_sync(0xffffffffu, resc)) {
-        // this half rescales its half of the O columns
 #pragma unroll
-        for (int q = 0; q < C / 64; ++q) {
+        for (int q = 0; q < C / 32; ++q) {
           float o[32];
-          const uint32_t ta = tO + lane_off + half * (C / 2) + q * 32;
-          tmem_ld32(ta, o);
+          tmem_ld32(tOg + q * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= corr;
-          tmem_st32(ta, o);
+          tmem_st32(tOg + q * 32, o);
         }
         tmem_wait_st();
       }
-      // P half row -> shared memory region `half`, 128-byte swizzled K-major
+      // P_g half row -> shared memory region g, 128-byte swizzled K-major
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint4 v;
@@ -323,55 +348,61 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         v.y = pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]);
         v.z = pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]);
         v.w = pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]);
-        const uint32_t addr = sP + half * L::kRegion + q_row * 128 + ((ch ^ (q_row & 7)) << 4);
+        const uint32_t addr = sP + g * L::kRegion + q_row * 128 + ((ch ^ (q_row & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                      "r"(v.z), "r"(v.w) : "memory");
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[g]);
       ++j;
     }
 
-    // epilogue: the row sum is the two halves' shares; each half normalises and
-    // writes its half of the O columns; lse = (m + log2 l) ln 2
-    if (ok) {
-      xsum[half * 128 + q_row] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(l_full);
-      ok = __all_sync(0xffffffffu, mbar_wait(l_full, 0, abort_flag));
-    }
-    const float lt = ok ? xsum[q_row] + xsum[128 + q_row] : 0.f;
-    bf16* orow = O + ((size_t)bh * M + (size_t)r * 128 + q_row) * C + half * (C / 2);
+    // last PV of this half, then merge the halves: publish (m_g, l_g)
     if (ok && j > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
-      if (ok) {
-        tc_fence_after();
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[g], (j - 1) & 1, abort_flag));
+    }
+    if (ok) {
+      xchg[g * 128 + q_row] = make_float2(m, l);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_full);
+      ok = __all_sync(0xffffffffu, mbar_wait(x_full, 0, abort_flag));
+    }
+    if (ok) {
+      tc_fence_after();   // the other half's last PV completed before it arrived
+      const float2 s0 = xchg[q_row], s1 = xchg[128 + q_row];
+      const bool has0 = s0.y > 0.f, has1 = s1.y > 0.f;
+      const float mm = fmaxf(has0 ? s0.x : kNegInf, has1 ? s1.x : kNegInf);
+      const float f0 = has0 ? ex2(s0.x - mm) : 0.f;
+      const float f1 = has1 ? ex2(s1.x - mm) : 0.f;
+      const float lt = s0.y * f0 + s1.y * f1;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      // this half writes output columns [g*C/2, (g+1)*C/2)
+      bf16* orow = O + ((size_t)bh * M + (size_t)r * 128 + q_row) * C + g * (C / 2);
+      const uint32_t tO0 = tmem + lane_off + L::kColO + g * (C / 2);
 #pragma unroll
-        for (int q = 0; q < C / 64; ++q) {
-          float o[32];
-          tmem_ld32(tO + lane_off + half * (C / 2) + q * 32, o);
-          tmem_wait_ld();
+      for (int q = 0; q < C / 64; ++q) {
+        float a0[32], a1[32];
+        tmem_ld32(tO0 + q * 32, a0);
+        tmem_ld32(tO0 + 128 + q * 32, a1);
+        tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 v;
-            v.x = pack_bf16x2(o[i + 0] * inv, o[i + 1] * inv);
-            v.y = pack_bf16x2(o[i + 2] * inv, o[i + 3] * inv);
-            v.z = pack_bf16x2(o[i + 4] * inv, o[i + 5] * inv);
-            v.w = pack_bf16x2(o[i + 6] * inv, o[i + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
-          }
+        for (int i = 0; i < 32; i += 8) {
+          float vv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            vv[e] = ((has0 ? a0[i + e] * f0 : 0.f) + (has1 ? a1[i + e] * f1 : 0.f)) * inv;
+          uint4 v;
+          v.x = pack_bf16x2(vv[0], vv[1]);
+          v.y = pack_bf16x2(vv[2], vv[3]);
+          v.z = pack_bf16x2(vv[4], vv[5]);
+          v.w = pack_bf16x2(vv[6], vv[7]);
+          *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
         }
-        if (lse != nullptr && half == 0)
-          lse[(size_t)bh * M + (size_t)r * 128 + q_row] = lt > 0.f ? (m + lg2(lt)) * kLn2 : kNegInf;
       }
-    } else if (ok && j == 0) {
-      const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int i = 0; i < C / 2; i += 8) *reinterpret_cast<uint4*>(orow + i) = z;
-      if (lse != nullptr && half == 0) lse[(size_t)bh * M + (size_t)r * 128 + q_row] = kNegInf;
+      if (lse != nullptr && g == 0)
+        lse[(size_t)bh * M + (size_t)r * 128 + q_row] = lt > 0.f ? (mm + lg2(lt)) * kLn2 : kNegInf;
     }
     tc_fence_before();
   }

@@ -88,7 +88,7 @@ int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
                     int diagonal, float scale, float* scores, float* part, float* lse_ws,
                     cudaStream_t st) {
 #ifndef XATTN_SCORE_BN
-#define XATTN_SCORE_BN 128
+#define XATTN_SCORE_BN 256
 #endif
   constexpr int BN = XATTN_SCORE_BN;
   auto kern = score_tc_kernel<C, G, BN>;

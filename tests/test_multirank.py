@@ -1,0 +1,55 @@
+"""The multi-rank host logic of bench.py on CPU (gloo, world size 2): the job time
+is the max over ranks, the whole-job metric divides by every rank's layers, and
+the reference arm runs on rank 0 only."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import synthetic as sy
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local_ms = 100.0 + 10.0 * rank          # rank 1 is the slow one
+        total = bench.dist_max(local_ms, dist, torch.device("cpu"))
+        out[rank] = (total, bench.job_ms_per_layer(total, steps=5, world=world, batch=1))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_is_max_over_ranks():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 110.0
+    assert res[0][1] == pytest.approx(110.0 / (5 * 2))
+
+
+def test_single_rank_helpers():
+    assert bench.dist_max(3.5) == 3.5
+    assert bench.job_ms_per_layer(50.0, steps=5, world=1, batch=2) == 5.0
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    class A:
+        seed, steps, warmup, cpu_seconds, gpus = 1, 1, 0, 0.1, 2
+    w = sy.workload("tiny_1h_2k")
+    assert bench.reference_arm(A, w, rank=1, world=2) == 0
+    assert capsys.readouterr().out == ""
