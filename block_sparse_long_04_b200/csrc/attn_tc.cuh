@@ -8,10 +8,15 @@
 //   warp 0, one lane  TMA producer: Q once, then the K and V tiles of the kept
 //                     blocks (in list order) into two rings of kStages stages with
 //                     their own full/empty barriers; K runs one block ahead of V.
-//   warp 1, one lane  MMA issuer and TMEM owner: S = Q K^T into TMEM (128 lanes x
+//   warp 1, one lane  S issuer and TMEM owner: S = Q K^T into TMEM (128 lanes x
 //                     128 fp32 columns); S of block j+1 is issued as soon as the
-//                     softmax has read S of block j. Then, per key half g (keys
-//                     64g..64g+63), O_g += P_g V_g into its own TMEM accumulator.
+//                     softmax has read S of block j.
+//   warp 2, one lane  PV issuer: per key half g (keys 64g..64g+63), O_g += P_g V_g
+//                     into its own TMEM accumulator. Issuing is split over two
+//                     threads on different sub-partitions because one thread
+//                     cannot issue the 16 MMAs of a block and poll their barriers
+//                     as fast as the tensor core retires them; each issuer's
+//                     commits track exactly its own MMAs.
 //   warps 4-11        softmax, two threads per query row (TMEM lane = row): warps
 //                     4-7 own keys 0-63 of every block, warps 8-11 keys 64-127.
 //                     The two halves are independent online softmaxes over
@@ -110,9 +115,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* s_free = q_full + 2;      // all 8 softmax warps have read it
   uint64_t* p_full = q_full + 3;      // [2] P_g written (4 warps each)
   uint64_t* o_done = q_full + 5;      // [2] PV_g of the block completed
-  uint64_t* drain = q_full + 7;
-  uint64_t* x_full = q_full + 8;      // end-of-row (m_g, l_g) published (8 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 9);
+  uint64_t* drain = q_full + 7;       // [2] S issuer, PV issuer
+  uint64_t* x_full = q_full + 9;      // end-of-row (m_g, l_g) published (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* xchg = reinterpret_cast<float2*>(smem + L::kOffX);   // [2 half][128]
 
@@ -136,7 +141,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(s_free, 8);
     mbar_init(&p_full[0], 4); mbar_init(&p_full[1], 4);
     mbar_init(&o_done[0], 1); mbar_init(&o_done[1], 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1); mbar_init(&drain[1], 1);
     mbar_init(x_full, 8);
     *abort_flag = 0;
     fence_mbar_init();
@@ -203,63 +208,72 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int jj = (nv > ST ? nv - ST : 0); jj < nv; ++jj)
         mbar_wait(&v_full[jj % ST], (jj / ST) & 1, &no_abort);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------- S and PV issuers
     if (lane == 0) {
+      // descriptors built once; per MMA only the start address (16-byte units,
+      // low bits) moves, which never carries out of its 14-bit field here
+      const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sK0, 16, 1024);
+      const uint64_t dP = smem_desc_sw128(sP, 16, 1024);
+      const uint64_t dV = smem_desc_sw128(sV0, L::kRegion, 1024);
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, C, false, true);
-      auto issue_S = [&](int j) {
-        const int st = j % ST;
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kRegion + (kk & 3) * 32;
-          mma_f16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024),
-                     smem_desc_sw128(sK0 + st * L::kTile + off, 16, 1024), idS, kk > 0);
-        }
-        mma_commit(s_full);
-        mma_commit(&k_empty[st]);
-      };
       ListIter li;
       li.init(col_idx, beg, end, nb, r, causal != 0, DENSE);
       bool have_cur = li.next() >= 0;
       bool have_nxt = have_cur && li.next() >= 0;
-      bool ok = have_cur && mbar_wait(q_full, 0, abort_flag);
-      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_S(0);
-      }
-      for (int j = 0; ok && have_cur; ++j) {
-        const int st = j % ST;
-        if (have_nxt) {
+      bool ok = true;
+      if (warp == 1) {
+        auto issue_S = [&](int j) {
+          const int st = j % ST;
+          const uint64_t dKs = dK + (uint64_t)((st * L::kTile) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * L::kRegion + (kk & 3) * 32) >> 4;
+            mma_f16_ss(tS, dQ + off, dKs + off, idS, kk > 0);
+          }
+          mma_commit(s_full);
+          mma_commit(&k_empty[st]);
+        };
+        ok = have_cur && mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_S(0);
+        }
+        for (int j = 0; ok && have_nxt; ++j) {
           ok = mbar_wait(&k_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag) &&
                mbar_wait(s_free, j & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_S(j + 1);
+          have_nxt = li.next() >= 0;
         }
-        if (!(ok = mbar_wait(&v_full[st], (j / ST) & 1, abort_flag))) break;
-        for (int g = 0; g < 2; ++g) {
-          if (!(ok = mbar_wait(&p_full[g], j & 1, abort_flag))) break;
-          tc_fence_after();
+      } else {
+        for (int j = 0; ok && have_cur; ++j) {
+          const int st = j % ST;
+          if (!(ok = mbar_wait(&v_full[st], (j / ST) & 1, abort_flag))) break;
+          for (int g = 0; g < 2; ++g) {
+            if (!(ok = mbar_wait(&p_full[g], j & 1, abort_flag))) break;
+            tc_fence_after();
+            const uint64_t dPg = dP + (uint64_t)((g * L::kRegion) >> 4);
+            const uint64_t dVg = dV + (uint64_t)((st * L::kTile + g * 4 * 2048) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {   // keys 64g + 16kk .. +15
-            mma_f16_ss(tmem + L::kColO + g * 128,
-                       smem_desc_sw128(sP + g * L::kRegion + kk * 32, 16, 1024),
-                       smem_desc_sw128(sV0 + st * L::kTile + (g * 4 + kk) * 2048, L::kRegion, 1024),
-                       idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)     // keys 64g + 16kk .. +15
+              mma_f16_ss(tmem + L::kColO + g * 128, dPg + (kk * 32 >> 4), dVg + (kk * 2048 >> 4),
+                         idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&o_done[g]);
           }
-          mma_commit(&o_done[g]);
+          if (!ok) break;
+          mma_commit(&v_empty[st]);
+          have_cur = have_nxt;
+          have_nxt = have_cur && li.next() >= 0;
         }
-        if (!ok) break;
-        mma_commit(&v_empty[st]);
-        have_cur = have_nxt;
-        have_nxt = have_cur && li.next() >= 0;
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
-      mma_commit(drain);
+      mma_commit(&drain[warp - 1]);
       volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort);
+      mbar_wait(&drain[warp - 1], 0, &no_abort);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
