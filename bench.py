@@ -60,6 +60,32 @@ def workload_of(a):
     return w.with_(stride=a.stride) if a.stride else w
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama8b_gqa_128k.json")
+KERNEL_SOURCES = {"attn_tc": ["attn_tc.cuh"], "score_tc": ["score_tc.cuh"]}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "block_sparse_long_04_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, workload: str, stride: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None
+    when there is none for this workload or the kernel's sources changed since."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    k = d.get("kernels", {}).get(kernel)
+    if (k is None or d.get("workload") != workload or d.get("stride") != stride
+            or k.get("source_sha256") != kernel_source_hash(kernel)):
+        return None
+    return k["dram_bytes_read"] + k["dram_bytes_write"]
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -299,7 +325,7 @@ def main():
                 "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": attn_tflops / pk["bf16_sustained"],
                 "peak_source": f"{pk['source']} bf16 sustained (kernel runs inside a long step)",
-                "traffic": None,
+                "traffic": measured_traffic("attn_tc", w.name, w.stride),
                 "algorithmic": "4*b^2*C FLOP per kept (head, query block, key block), "
                                "diagonal blocks counted in full"}
     score_flops = (1.0 if w.causal else 2.0) * w.M * w.M * C * w.Hq * w.B / w.stride

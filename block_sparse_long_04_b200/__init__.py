@@ -45,6 +45,7 @@ SIGNATURES = {
     "xattn_select_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _Z, _P, _P]),
     "xattn_score_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _Z, _P]),
     "xattn_select_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
+    "xattn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _P, _P]),
 }
 
 XATTN_PATTERN_ANTIDIAGONAL, XATTN_PATTERN_DIAGONAL = 0, 1
@@ -210,6 +211,14 @@ def xattn_dense_attn(Q, K, V, causal: bool, softmax_scale: float, O, lse=None, b
     rc = _lib.xattn_dense_attn(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, M, C, block, int(causal),
                                float(softmax_scale), _ptr(O), _ptr(lse), _stream(stream))
     _check(rc, "xattn_dense_attn")
+
+
+def xattn_selftest_wait_timeout(limit_ns: int, timed_out, stream=None) -> None:
+    """Diagnostic: a device wait that nothing completes must give up after
+    limit_ns and raise XATTN_ETIMEOUT (read it with xattn_get_device_error)."""
+    _dev(timed_out)
+    _check(_lib.xattn_selftest_wait_timeout(int(limit_ns), _ptr(timed_out), _stream(stream)),
+           "xattn_selftest_wait_timeout")
 
 
 def xattn_get_device_error(stream=None) -> int:

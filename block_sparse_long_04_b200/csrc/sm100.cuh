@@ -41,9 +41,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Gives up after
-// kWaitLimitNs, or as soon as another thread of the CTA has given up (*abort),
-// in which case it raises XATTN_ETIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// limit_ns, or as soon as another thread of the CTA has given up (*abort), in
+// which case it raises XATTN_ETIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
@@ -53,11 +54,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       raise_device_error(kErrTimeout);
       return false;
     }
+  }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
+}
+
+// Diagnostic: waits on an mbarrier that nothing arrives at, for at most
+// limit_ns; the wait must end with XATTN_ETIMEOUT in the device error word and
+// *result = 1 (timed out). Exercises the bounded-wait path without any copy or
+// tensor-core work in flight.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, int* result) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait_for(&bar, 0, &abort_flag, limit_ns);
+    *result = ok ? 0 : 1;
   }
 }
 

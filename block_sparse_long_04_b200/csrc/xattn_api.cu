@@ -361,6 +361,13 @@ int xattn_dense_attn(const void* Q, const void* K, const void* V, int B, int Hq,
                            softmax_scale, O, lse, stream);
 }
 
+int xattn_selftest_wait_timeout(long long limit_ns, int32_t* timed_out, void* stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000LL || timed_out == nullptr) return XATTN_EINVAL;
+  sm100::wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(
+      (unsigned long long)limit_ns, timed_out);
+  return launch_status();
+}
+
 int xattn_get_device_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return XATTN_ECUDA;
   int v = 0;

@@ -250,6 +250,16 @@ XATTN_API int xattn_dense_attn(const void* Q, const void* K, const void* V,
                      float softmax_scale, void* O, float* lse, void* stream);
 
 /*
+ * xattn_selftest_wait_timeout - diagnostic of the bounded device waits (the
+ * pages have no counterpart). Launches one CTA that waits on a barrier nothing
+ * will ever complete, for at most limit_ns nanoseconds (1 .. 1e9). The wait must
+ * give up, raise XATTN_ETIMEOUT in the device error word and write 1 to
+ * *timed_out (int32, device memory). The context stays usable; read the status
+ * with xattn_get_device_error. Limits outside the range return XATTN_EINVAL.
+ */
+XATTN_API int xattn_selftest_wait_timeout(long long limit_ns, int32_t* timed_out, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's error
  * word (XATTN_OK if no device-side condition was raised since the last call).
  * Returns XATTN_ECUDA if the synchronisation itself failed.

@@ -175,3 +175,9 @@ def test_unknown_pattern_and_rule_are_rejected():
     rc = xa._lib.xattn_score_ex(FAKE, FAKE, 1, 4, 2, 1000, 128, 8, 128, 1, 1, 0.03, FAKE, FAKE,
                                 1 << 40, None)
     assert rc == xa.XATTN_EINVAL   # M not a multiple of the block
+
+
+def test_selftest_rejects_bad_limits():
+    for bad in (0, -5, 2_000_000_000):
+        assert xa._lib.xattn_selftest_wait_timeout(bad, FAKE, None) == xa.XATTN_EINVAL
+    assert xa._lib.xattn_selftest_wait_timeout(1000, None, None) == xa.XATTN_EINVAL
