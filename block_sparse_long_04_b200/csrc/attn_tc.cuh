@@ -28,8 +28,8 @@
 //                     Per block: read the half row of S, causal mask on the
 //                     diagonal block, fp32 base-2 softmax with the scale folded into
 //                     one FMA, lazy rescaling (O_g and l_g are rescaled only when
-//                     m_g grows by more than 2^8), P_g as bf16 into shared memory in
-//                     the tensor core's 128-byte-swizzled K-major layout.
+//                     m_g grows by more than 2^8), P_g as bf16 into TMEM, where the
+//                     PV MMA reads it as its A operand.
 // Every role walks the row's list with the next entry's load already in flight
 // (ListIter), so no role waits on a global load inside its loop.
 // Every wait is bounded (sm100::mbar_wait); on a timeout the CTA raises
@@ -52,13 +52,13 @@ struct AttnTc {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffP = kOffV + kStages * kTile;   // 128 x 128 bf16, region g = half g
-  static constexpr int kOffBar = kOffP + 2 * kRegion;
+  static constexpr int kOffBar = kOffV + kStages * kTile;
   static constexpr int kOffX = kOffBar + 256;             // end-of-row (m, l) exchange
   static constexpr int kSmem = kOffX + 2 * 128 * 8 + 1024;  // + alignment slack
-  static constexpr int kTmemCols = 512;                   // S 0..127, O_0 128.., O_1 256..
-  static constexpr int kColS = 0;
-  static constexpr int kColO = 128;                       // + g * 128
+  static constexpr int kTmemCols = 512;                   // S, O_0, O_1, P_0, P_1
+  static constexpr int kColS = 0;                         // 128 fp32 columns
+  static constexpr int kColO = 128;                       // + g * 128: C fp32 columns each
+  static constexpr int kColP = 384;                       // + g * 32: 64 bf16 keys each
 };
 
 // Walks the kept-block list of one row, skipping entries outside [0, nb) and,
@@ -104,7 +104,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t sQ = smem_u32(smem + L::kOffQ);
   const uint32_t sK0 = smem_u32(smem + L::kOffK);
   const uint32_t sV0 = smem_u32(smem + L::kOffV);
-  const uint32_t sP = smem_u32(smem + L::kOffP);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* k_full = bars;            // [ST] K tile of a block landed
   uint64_t* k_empty = bars + ST;      // [ST] its S MMA completed
@@ -215,7 +214,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // low bits) moves, which never carries out of its 14-bit field here
       const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dK = smem_desc_sw128(sK0, 16, 1024);
-      const uint64_t dP = smem_desc_sw128(sP, 16, 1024);
       const uint64_t dV = smem_desc_sw128(sV0, L::kRegion, 1024);
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, C, false, true);
@@ -256,12 +254,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int g = 0; g < 2; ++g) {
             if (!(ok = mbar_wait(&p_full[g], j & 1, abort_flag))) break;
             tc_fence_after();
-            const uint64_t dPg = dP + (uint64_t)((g * L::kRegion) >> 4);
             const uint64_t dVg = dV + (uint64_t)((st * L::kTile + g * 4 * 2048) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)     // keys 64g + 16kk .. +15
-              mma_f16_ss(tmem + L::kColO + g * 128, dPg + (kk * 32 >> 4), dVg + (kk * 2048 >> 4),
-                         idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)     // keys 64g + 16kk .. +15 (8 TMEM columns)
+              mma_f16_ts(tmem + L::kColO + g * 128, tmem + L::kColP + g * 32 + kk * 8,
+                         dVg + (kk * 2048 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&o_done[g]);
           }
           if (!ok) break;
@@ -282,6 +279,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tSg = tS + lane_off + g * 64;
     const uint32_t tOg = tmem + lane_off + L::kColO + g * 128;
+    const uint32_t tPg = tmem + lane_off + L::kColP + g * 32;
     const int k0 = g * 64;
     float m = kNegInf, l = 0.f;
     int j = 0;
@@ -354,19 +352,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         tmem_wait_st();
       }
-      // P_g half row -> shared memory region g, 128-byte swizzled K-major
+      // P_g half row -> TMEM (A operand of the PV MMA): 64 bf16 keys packed two
+      // per 32-bit column, one store per thread
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint4 v;
-        v.x = pack_bf16x2(s[ch * 8 + 0], s[ch * 8 + 1]);
-        v.y = pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]);
-        v.z = pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]);
-        v.w = pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]);
-        const uint32_t addr = sP + g * L::kRegion + q_row * 128 + ((ch ^ (q_row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                     "r"(v.z), "r"(v.w) : "memory");
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+        tmem_st32(tPg, reinterpret_cast<const float*>(pk));
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[g]);
