@@ -293,3 +293,35 @@ def test_empty_problem_is_a_no_op():
     ws = torch.empty(16, dtype=torch.uint8, device="cuda")
     xa.xattn_score(Q, Q[:, :1], 8, True, 0.1, scores, ws)
     assert xa.xattn_get_device_error() == xa.XATTN_OK
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_batch_of_two_layers(causal):
+    """B = 2: every kernel indexes (batch, head) rows, KV heads and CSR rows by
+    batch; each batch element must match the oracle on its own inputs."""
+    w = small_workload(1536, 128, 4, 2, 8, causal).with_(B=2)
+    (Qb, Kb, Vb), (Q, K, V) = device_inputs(w)
+    tau = np.array([0.9, 0.8, 0.95, 0.7], np.float32)
+    bufs = _pipeline(w, Q, K, V, tau, with_lse=True)
+    nb = w.nb
+    ref_s = _oracle_scores(Qb, Kb, w)
+    got_s = bufs.scores.cpu().numpy()
+    row_ptr, col = bufs.row_ptr.cpu().numpy(), bufs.col_idx.cpu().numpy()
+    fails = []
+    kept_gpu = {}
+    for b in range(2):
+        for h in range(w.Hq):
+            P.assert_scores_close(got_s[b, h], ref_s[(b, h)], f"scores b{b} h{h}")
+            bh = b * w.Hq + h
+            kept_gpu[(b, h)] = csr_to_dict(row_ptr, col, bh, nb)
+            for r in range(nb):
+                _, f = P.compare_row_mask(kept_gpu[(b, h)][r], ref_s[(b, h)][r], r, float(tau[h]),
+                                          causal)
+                fails += f
+    assert not fails, fails[:5]
+    ref_o = orc.layer_sparse_attention(Qb, Kb, Vb, w.Hkv, kept_gpu, 128, causal, 1 / math.sqrt(w.C))
+    got_o = bf16_to_np(bufs.O)
+    got_l = bufs.lse.cpu().numpy()
+    for (b, h), (o, l) in ref_o.items():
+        P.assert_outputs_close(got_o[b, h], o, f"O b{b} h{h}")
+        np.testing.assert_allclose(got_l[b, h], l, rtol=1e-4, atol=1e-4)
