@@ -305,14 +305,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int i = 0; i < 64; ++i) s[i] = (k0 + i > q_row) ? kNegInf : s[i];
       }
       // eight independent partial maxima / sums keep the reductions off one
-      // long dependency chain
+      // long dependency chain; three-input max and packed fp32x2 FMA / add halve
+      // the instruction count of the two reductions and of the exponent arguments
       float pm[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) pm[k] = s[k];
 #pragma unroll
-      for (int i = 8; i < 64; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      for (int i = 8; i < 64; i += 2) pm[(i >> 1) & 7] = fmax3(pm[(i >> 1) & 7], s[i], s[i + 1]);
+      const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]),
+                             fmaxf(pm[6], pm[7]));
       // a row may see no key of this half (the upper half of the diagonal block)
       const float m_new = fmaxf(m, mx * scale_log2);
       float corr = 1.f;
@@ -325,13 +326,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         resc = true;
       }
       const float neg_m = (m == kNegInf) ? 0.f : -m;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
+      float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = ex2(fmaf(s[i], scale_log2, neg_m));
-        ps[i & 7] += s[i];
+      for (int i = 0; i < 64; i += 2) {
+        const float2 x = ffma2(make_float2(s[i], s[i + 1]), sc2, nm2);
+        s[i] = ex2(x.x);
+        s[i + 1] = ex2(x.y);
+        ps[(i >> 1) & 3] = fadd2(ps[(i >> 1) & 3], make_float2(s[i], s[i + 1]));
       }
-      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      const float2 pq = fadd2(fadd2(ps[0], ps[1]), fadd2(ps[2], ps[3]));
+      const float rs = pq.x + pq.y;
       l = l * corr + rs;
 
       // PV_g of the previous block must be complete: P_g free, O_g stable

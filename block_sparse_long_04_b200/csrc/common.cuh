@@ -69,6 +69,30 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// max of three fp32 values in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// packed fp32x2 arithmetic (two lanes per instruction, sm_100)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long ua, ub, uc, ud;
+  ua = *reinterpret_cast<unsigned long long*>(&a);
+  ub = *reinterpret_cast<unsigned long long*>(&b);
+  uc = *reinterpret_cast<unsigned long long*>(&c);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ud) : "l"(ua), "l"(ub), "l"(uc));
+  return *reinterpret_cast<float2*>(&ud);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  unsigned long long ua, ub, ud;
+  ua = *reinterpret_cast<unsigned long long*>(&a);
+  ub = *reinterpret_cast<unsigned long long*>(&b);
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(ud) : "l"(ua), "l"(ub));
+  return *reinterpret_cast<float2*>(&ud);
+}
+
 // Byte offset of 16-byte chunk `ch` of row `row` in a tile whose rows are
 // `row_bytes` long, XOR-swizzled on the low three chunk bits so that eight
 // consecutive rows at the same logical chunk hit eight different bank groups.
