@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fused-select", action="store_true",
+                    help="score and select in the one fused call instead of two calls")
     return ap.parse_args()
 
 
@@ -274,11 +276,20 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        xa.xattn_score(Q, K, w.stride, w.causal, ss, bufs.scores, bufs.score_ws, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        xa.xattn_select(bufs.scores, tau, w.causal, bufs.row_ptr, bufs.col_idx, bufs.nnz,
-                        bufs.select_ws, stream=stream)
+        if not a.fused_select:
+            xa.xattn_score(Q, K, w.stride, w.causal, ss, bufs.scores, bufs.score_ws,
+                           stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            xa.xattn_select(bufs.scores, tau, w.causal, bufs.row_ptr, bufs.col_idx, bufs.nnz,
+                            bufs.select_ws, stream=stream)
+        else:
+            # scoring kernel ranks and cuts each row; then the scan and fill passes
+            xa.xattn_score_select(Q, K, tau, xa.XATTN_SELECT_THRESHOLD, w.stride, w.causal, ss,
+                                  bufs.scores, bufs.row_ptr, bufs.col_idx, bufs.nnz,
+                                  bufs.score_ws, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
         if ev is not None:
             ev[2].record(stream)
         xa.xattn_sparse_attn(Q, K, V, bufs.row_ptr, bufs.col_idx, w.causal, sa, bufs.O,
@@ -286,7 +297,9 @@ def main():
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 5   # score 1, select 3, sparse attention 1
+    # unfused: score 1, select 3 (count, scan, fill), attention 1;
+    # fused: score with row cuts 1, scan 1, fill 1, attention 1
+    launches_per_step = 4 if a.fused_select else 5
     for _ in range(a.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -330,11 +343,14 @@ def main():
                                "diagonal blocks counted in full"}
     score_flops = (1.0 if w.causal else 2.0) * w.M * w.M * C * w.Hq * w.B / w.stride
     extra = {
-        "stages_ms": {"score": st_score, "select": st_select, "sparse_attn": st_attn},
+        "stages_ms": ({"score": st_score, "select": st_select, "sparse_attn": st_attn}
+                      if not a.fused_select else
+                      {"score_select": st_score + st_select, "sparse_attn": st_attn}),
         "density": density, "nnz": nnz,
         "kept_block_tflops": attn_tflops,
         "kept_block_frac_of_bf16_peak": attn_tflops / pk["bf16_sustained"],
         "dense_equivalent_tflops": dense_eq_flops / (ms_step * 1e-3) / 1e12,
+        # fused: the score stage also holds the row ranking, scan and fill
         "score_tflops": score_flops / (st_score * 1e-3) / 1e12,
     }
 

@@ -46,6 +46,9 @@ SIGNATURES = {
     "xattn_score_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _Z, _P]),
     "xattn_select_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
     "xattn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _P, _P]),
+    "xattn_score_select_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "xattn_score_select": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _Z,
+                                _P, _P, _Z, _P]),
 }
 
 XATTN_PATTERN_ANTIDIAGONAL, XATTN_PATTERN_DIAGONAL = 0, 1
@@ -163,6 +166,26 @@ def xattn_select_ex(scores, param, rule: int, causal: bool, row_ptr, col_idx, nn
     _check(rc, "xattn_select_ex")
 
 
+def xattn_score_select_workspace_size(B: int, Hq: int, M: int, stride: int, block: int = 128) -> int:
+    return int(_lib.xattn_score_select_workspace_size(B, Hq, M, stride, block))
+
+
+def xattn_score_select(Q, K, param, rule: int, stride: int, causal: bool, score_scale: float, scores,
+                       row_ptr, col_idx, nnz, workspace, block: int = 128, stream=None) -> None:
+    """Scores and kept lists in one fused pass (same results as xattn_score followed
+    by xattn_select_ex)."""
+    _dev(Q, K, param, scores, row_ptr, col_idx, nnz, workspace)
+    _bf16(Q, K)
+    B, Hq, M, C = Q.shape
+    Hkv = K.shape[1]
+    rc = _lib.xattn_score_select(_ptr(Q), _ptr(K), B, Hq, Hkv, M, C, stride, block, int(causal),
+                                 float(score_scale), _ptr(param), int(rule), _ptr(scores),
+                                 _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(nnz),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(rc, "xattn_score_select")
+
+
 def xattn_select(scores, tau, causal: bool, row_ptr, col_idx, nnz, workspace, stream=None) -> None:
     """CSR (row_ptr, col_idx, nnz) <- per-head threshold selection of scores."""
     _dev(scores, tau, row_ptr, col_idx, nnz, workspace)
@@ -251,7 +274,8 @@ class Buffers:
         cap = max_kept(B, Hq, nb, causal) if col_capacity is None else col_capacity
         return Buffers(
             scores=torch.empty((B, Hq, nb, nb), dtype=torch.float32, device=dev),
-            score_ws=torch.empty(max(1, xattn_score_workspace_size(B, Hq, M, stride, block)),
+            # sized for the fused score+select call, which also serves xattn_score
+            score_ws=torch.empty(max(1, xattn_score_select_workspace_size(B, Hq, M, stride, block)),
                                  dtype=torch.uint8, device=dev),
             select_ws=torch.empty(max(1, xattn_select_workspace_size(B, Hq, nb)),
                                   dtype=torch.uint8, device=dev),
@@ -271,7 +295,11 @@ def default_score_scale(stride: int, C: int) -> float:
 def xattn_prefill(Q, K, V, tau, stride: int, causal: bool, bufs: Buffers,
                   score_scale: Optional[float] = None, softmax_scale: Optional[float] = None,
                   block: int = 128, stream=None) -> torch.Tensor:
-    """score -> select -> sparse attention on one stream; returns bufs.O."""
+    """score -> select -> sparse attention on one stream; returns bufs.O.
+
+    Scoring and selection run as two calls: on B200 that is faster than the fused
+    xattn_score_select, whose in-kernel ranking runs on one CTA per SM behind the
+    scoring tile."""
     C = Q.shape[-1]
     ss = default_score_scale(stride, C) if score_scale is None else score_scale
     sa = 1.0 / math.sqrt(C) if softmax_scale is None else softmax_scale

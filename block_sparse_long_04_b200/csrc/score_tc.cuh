@@ -26,8 +26,14 @@
 // CTA's ell values (L2-resident) and write
 //   scores[r, c] = (1/g) sum_{i' in r} 2^(ell[i', c] - LSE[i']).
 // The (M/S)^2 logits are never stored. Waits are bounded as in attn_tc.cuh.
+//
+// With SELECT set (the fused score -> select path), the same 128 threads then run
+// the threshold selection of every query-block row they have just finished
+// (select.cuh, select_row_cut) in the now idle stage ring, and record each row's
+// cut, so that the selection needs only its scan and fill passes afterwards.
 #pragma once
 #include "common.cuh"
+#include "select.cuh"
 #include "sm100.cuh"
 
 namespace xattn {
@@ -42,15 +48,26 @@ struct ScoreTc {
   static constexpr int kStageBytes = kQBytes + kKBytes;
   static constexpr int kOffBar = kStages * kStageBytes;
   static constexpr int kOffLse = kOffBar + 256;
-  static constexpr int kSmem = kOffLse + 128 * 4 + 1024;
+  static constexpr int kSmem = kOffLse + 128 * 4 + 16 + 1024;
   static constexpr int kTmemCols = 2 * BN;
 };
 
-template <int C, int G, int BN>
+template <int C, int G, int BN, bool SELECT>
 __global__ void __launch_bounds__(kScoreTcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 int Hq, int Hkv, int M, int causal, int diagonal, float scale_log2,
-                float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores) {
+                float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores,
+                const float* __restrict__ sel_param, int sel_rule, SelCut* __restrict__ cuts);
+
+static_assert(ScoreTc<128>::kOffBar >= kSelMaxNb * 8 + 64 && ScoreTc<256>::kOffBar >= kSelMaxNb * 8 + 64,
+              "the stage ring must hold the fused selection's sort keys");
+
+template <int C, int G, int BN, bool SELECT>
+__global__ void __launch_bounds__(kScoreTcThreads, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                int Hq, int Hkv, int M, int causal, int diagonal, float scale_log2,
+                float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores,
+                const float* __restrict__ sel_param, int sel_rule, SelCut* __restrict__ cuts) {
   using L = ScoreTc<BN>;
   constexpr int ST = L::kStages;
   constexpr int S = 128 / G;
@@ -225,6 +242,33 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
           srow[c] = acc;
         }
+      }
+    }
+    if (SELECT) {
+      // fused selection of the rows just written; one uniform decision first
+      volatile int* go = reinterpret_cast<volatile int*>(lse_s + 128);
+      if (tid == 128) *go = (ok && !*abort_flag) ? 1 : 0;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*go) {
+        const int et = tid - 128;
+        float* key = reinterpret_cast<float*>(smem);                    // the idle stage ring
+        int* idx = reinterpret_cast<int*>(smem + kSelMaxNb * 4);
+        double* red = reinterpret_cast<double*>(smem + kSelMaxNb * 8);
+        int* first_hit = reinterpret_cast<int*>(red + 4);
+        auto sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+        for (int k = 0; k < 128 / G; ++k) {
+          const int r = i0 / G + k;
+          if (r >= nb) break;
+          const int n = causal ? r + 1 : nb;
+          const SelCut cut = select_row_cut<128>(scores + ((size_t)bh * nb + r) * nb, n, r,
+                                                 sel_param[h], sel_rule, key, idx, red,
+                                                 first_hit, et, sync);
+          if (et == 0) cuts[(size_t)bh * nb + r] = cut;
+        }
+      } else {
+        // no scores: empty cuts, so the scan and fill passes write nothing for these rows
+        const int r = i0 / G + (tid - 128);
+        if (tid - 128 < 128 / G && r < nb) cuts[(size_t)bh * nb + r] = SelCut{0.f, 0, 0};
       }
     }
     tc_fence_before();

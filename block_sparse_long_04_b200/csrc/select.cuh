@@ -41,32 +41,6 @@ __device__ __forceinline__ bool ranks_before(float sa, int ia, float sb, int ib)
   return sa > sb || (sa == sb && ia < ib);
 }
 
-__device__ __forceinline__ double block_exclusive_scan_f64(double v, double* red, double& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    double w = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    red[lane] = w;   // inclusive prefix of warp totals
-  }
-  __syncthreads();
-  const double before = (warp > 0 ? red[warp - 1] : 0.0) + (x - v);
-  total = red[(blockDim.x >> 5) - 1];
-  __syncthreads();
-  return before;
-}
-
 __device__ __forceinline__ int block_exclusive_scan_i32(int v, int* red, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
@@ -93,32 +67,48 @@ __device__ __forceinline__ int block_exclusive_scan_i32(int v, int* red, int& to
   return before;
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-select_count_kernel(const float* __restrict__ scores, const float* __restrict__ tau, int Hq, int nb,
-                    int causal, SelCut* __restrict__ cuts, int rule) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int row = blockIdx.x;
-  const int bh = row / nb, r = row % nb, h = bh % Hq;
-  const int n = causal ? r + 1 : nb;
+// Exclusive scan of one fp64 value per thread over a group of NT threads (whole
+// warps) that share `sync` as their barrier; red holds NT/32 doubles.
+template <int NT, typename Sync>
+__device__ __forceinline__ double group_exclusive_scan_f64(double v, double* red, int tid, Sync sync) {
+  const int lane = tid & 31, warp = tid >> 5;
+  double x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  sync();
+  double before = x - v;
+  for (int w = 0; w < warp; ++w) before += red[w];
+  sync();
+  return before;
+}
+
+// The cut of one row of block scores (candidates 0..n-1, diagonal r), computed
+// by a group of NT threads: bitonic sort of (score, index) keys in shared memory
+// (descending score, ascending index), then the cut position of the rule: the
+// first prefix whose fp64 cumulative sum reaches t (threshold), floor(t) (Top-K)
+// or ceil(t * n) (ratio), clamped to [1, n]. key/idx hold P floats / ints with
+// P = next power of two >= n. The result is valid in thread 0 of the group.
+template <int NT, typename Sync>
+__device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, float t, int rule,
+                                 float* key, int* idx, double* red, int* first_hit, int tid,
+                                 Sync sync) {
   int P = 1;
   while (P < n) P <<= 1;
-  float* key = reinterpret_cast<float*>(smem);
-  int* idx = reinterpret_cast<int*>(smem + (size_t)P * 4);
-  __shared__ double red[32];
-  __shared__ int first_hit;
-
-  const float* srow = scores + (size_t)row * nb;
-  for (int i = threadIdx.x; i < P; i += kSelThreads) {
+  for (int i = tid; i < P; i += NT) {
     key[i] = i < n ? srow[i] : kNegInf;
     idx[i] = i < n ? i : 0x7fffffff;
   }
-  if (threadIdx.x == 0) first_hit = n - 1;
-  __syncthreads();
+  if (tid == 0) *first_hit = n - 1;
+  sync();
 
   // bitonic network: ascending "rank" order = descending score, ascending index
   for (int k = 2; k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < P; i += kSelThreads) {
+      for (int i = tid; i < P; i += NT) {
         const int p = i ^ j;
         if (p > i) {
           const float si = key[i], sp = key[p];
@@ -131,44 +121,61 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
           }
         }
       }
-      __syncthreads();
+      sync();
     }
   }
 
-  const float t = tau[h];
   if (rule != kSelThreshold) {
     // Top-K / ratio: the cut position follows from the candidate count alone
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
       double kk = rule == kSelTopK ? floor((double)t) : ceil((double)t * (double)n);
       kk = kk < 1.0 ? 1.0 : (kk > (double)n ? (double)n : kk);   // NaN -> n
-      first_hit = (kk >= 1.0 && kk <= (double)n) ? (int)kk - 1 : n - 1;
+      *first_hit = (kk >= 1.0 && kk <= (double)n) ? (int)kk - 1 : n - 1;
     }
-    __syncthreads();
+    sync();
   }
   // fp64 prefix sums over contiguous per-thread segments of the sorted order
-
-  const int per = (n + kSelThreads - 1) / kSelThreads;
-  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  const int per = (n + NT - 1) / NT;
+  const int lo = tid * per, hi = min(n, lo + per);
   double seg = 0.0;
   for (int i = lo; i < hi; ++i) seg += (double)key[i];
-  double total;
-  double run = block_exclusive_scan_f64(seg, red, total);
+  double run = group_exclusive_scan_f64<NT>(seg, red, tid, sync);
   if (rule == kSelThreshold && t < 1.0f) {
     for (int i = lo; i < hi; ++i) {
       run += (double)key[i];
-      if (run >= (double)t) { atomicMin(&first_hit, i); break; }
+      if (run >= (double)t) { atomicMin(first_hit, i); break; }
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int k = first_hit;
-    const float cs = key[k];
-    const int ci = idx[k];
-    const bool diag_kept = ranks_before(srow[r], r, cs, ci) || (srow[r] == cs && r == ci);
-    cuts[row].score = cs;
-    cuts[row].index = ci;
-    cuts[row].count = k + 1 + (diag_kept ? 0 : 1);
+  sync();
+  SelCut cut;
+  if (tid == 0) {
+    const int k = *first_hit;
+    cut.score = key[k];
+    cut.index = idx[k];
+    const bool diag_kept = r == cut.index || ranks_before(srow[r], r, cut.score, cut.index);
+    cut.count = k + 1 + (diag_kept ? 0 : 1);
   }
+  sync();   // key/idx/first_hit may be reused by the caller's next row
+  return cut;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_count_kernel(const float* __restrict__ scores, const float* __restrict__ tau, int Hq, int nb,
+                    int causal, SelCut* __restrict__ cuts, int rule) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ double red[kSelThreads / 32];
+  __shared__ int first_hit;
+  const int row = blockIdx.x;
+  const int bh = row / nb, r = row % nb, h = bh % Hq;
+  const int n = causal ? r + 1 : nb;
+  int P = 1;
+  while (P < n) P <<= 1;
+  float* key = reinterpret_cast<float*>(smem);
+  int* idx = reinterpret_cast<int*>(smem + (size_t)P * 4);
+  const SelCut cut = select_row_cut<kSelThreads>(scores + (size_t)row * nb, n, r, tau[h], rule, key,
+                                                 idx, red, &first_hit, (int)threadIdx.x,
+                                                 [] { __syncthreads(); });
+  if (threadIdx.x == 0) cuts[row] = cut;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -214,7 +221,8 @@ select_fill_kernel(const float* __restrict__ scores, const SelCut* __restrict__ 
   for (int c = lo; c < hi; ++c) cnt += kept(c) ? 1 : 0;
   int total;
   int pos = block_exclusive_scan_i32(cnt, red, total);
-  for (int c = lo; c < hi; ++c)
+  // the row's count bounds the writes even if cuts and scores disagree
+  for (int c = lo; c < hi && pos < cut.count; ++c)
     if (kept(c)) col_idx[base + pos++] = c;
 }
 

@@ -83,15 +83,23 @@ int check_shape(int B, int Hq, int Hkv, int M, int C, int block) {
   return XATTN_OK;
 }
 
-template <int C, int G>
+// Optional fused selection of the scoring kernel: rule + per-head parameter, and
+// where to put each row's cut (null: scores only).
+struct FusedSelect {
+  const float* param = nullptr;
+  int rule = 0;
+  SelCut* cuts = nullptr;
+};
+
+template <int C, int G, bool SELECT>
 int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
                     int diagonal, float scale, float* scores, float* part, float* lse_ws,
-                    cudaStream_t st) {
+                    FusedSelect fs, cudaStream_t st) {
 #ifndef XATTN_SCORE_BN
 #define XATTN_SCORE_BN 256
 #endif
   constexpr int BN = XATTN_SCORE_BN;
-  auto kern = score_tc_kernel<C, G, BN>;
+  auto kern = score_tc_kernel<C, G, BN, SELECT>;
   constexpr int smem = ScoreTc<BN>::kSmem;
   static unsigned long long done = 0;
   if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
@@ -103,20 +111,21 @@ int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
     return XATTN_ECUDA;
   dim3 grid((rp + 127) / 128, B * Hq);
   kern<<<grid, kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, diagonal,
-                                            scale * kLog2e, part, lse_ws, scores);
+                                            scale * kLog2e, part, lse_ws, scores, fs.param,
+                                            fs.rule, fs.cuts);
   return launch_status();
 }
 
-template <int C>
+template <int C, bool SELECT>
 int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M,
                    int causal, int diagonal, float scale, float* scores, float* part,
-                   float* lse_ws, cudaStream_t st) {
+                   float* lse_ws, FusedSelect fs, cudaStream_t st) {
   switch (stride) {
-    case 1: return launch_score_tc<C, 128>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
-    case 2: return launch_score_tc<C, 64>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
-    case 4: return launch_score_tc<C, 32>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
-    case 8: return launch_score_tc<C, 16>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
-    case 16: return launch_score_tc<C, 8>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, st);
+    case 1: return launch_score_tc<C, 128, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
+    case 2: return launch_score_tc<C, 64, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
+    case 4: return launch_score_tc<C, 32, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
+    case 8: return launch_score_tc<C, 16, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
+    case 16: return launch_score_tc<C, 8, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
   }
   return XATTN_EUNSUPPORTED;
 }
@@ -164,6 +173,39 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_
                                     softmax_scale, o, lse, st);
 }
 
+template <bool SELECT = false>
+int score_common(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
+                        int stride, int block, int causal, int pattern, float score_scale,
+                        float* scores, void* workspace, size_t workspace_bytes, void* stream,
+                        FusedSelect fs = FusedSelect()) {
+  int rc = check_shape(B, Hq, Hkv, M, C, block);
+  if (rc != XATTN_OK) return rc;
+  if (stride <= 0 || block % stride != 0) return XATTN_EINVAL;
+  if (pattern != XATTN_PATTERN_ANTIDIAGONAL && pattern != XATTN_PATTERN_DIAGONAL)
+    return XATTN_EINVAL;
+  if (!stride_supported(stride)) return XATTN_EUNSUPPORTED;
+  if (B == 0 || Hq == 0 || M == 0) return XATTN_OK;
+  if (!Q || !K || !scores || !workspace) return XATTN_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace) || !aligned16(scores))
+    return XATTN_EINVAL;
+  if (!(score_scale > 0.f) || score_scale == __builtin_huge_valf()) return XATTN_EINVAL;
+  const size_t need = xattn_score_workspace_size(B, Hq, M, stride, block);
+  if (workspace_bytes < need) return XATTN_EINVAL;
+  const int rp = M / stride;
+  if ((rp + 127) / 128 > (1 << 30)) return XATTN_EUNSUPPORTED;
+  float* part = static_cast<float*>(workspace);
+  float* lse_ws = part + (size_t)B * Hq * rp * (M / block);
+  auto q = static_cast<const bf16*>(Q);
+  auto k = static_cast<const bf16*>(K);
+  cudaStream_t st = as_stream(stream);
+  const int diag = pattern == XATTN_PATTERN_DIAGONAL ? 1 : 0;
+  if (C == 64)
+    return launch_score_c<64, SELECT>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, diag,
+                                      score_scale, scores, part, lse_ws, fs, st);
+  return launch_score_c<128, SELECT>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, diag,
+                                     score_scale, scores, part, lse_ws, fs, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -187,37 +229,6 @@ size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block) {
     return 0;
   const size_t rp = (size_t)M / stride, nb = (size_t)M / block;
   return (size_t)B * Hq * rp * (nb + 1) * sizeof(float);
-}
-
-static int score_common(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
-                        int stride, int block, int causal, int pattern, float score_scale,
-                        float* scores, void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = check_shape(B, Hq, Hkv, M, C, block);
-  if (rc != XATTN_OK) return rc;
-  if (stride <= 0 || block % stride != 0) return XATTN_EINVAL;
-  if (pattern != XATTN_PATTERN_ANTIDIAGONAL && pattern != XATTN_PATTERN_DIAGONAL)
-    return XATTN_EINVAL;
-  if (!stride_supported(stride)) return XATTN_EUNSUPPORTED;
-  if (B == 0 || Hq == 0 || M == 0) return XATTN_OK;
-  if (!Q || !K || !scores || !workspace) return XATTN_EINVAL;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace) || !aligned16(scores))
-    return XATTN_EINVAL;
-  if (!(score_scale > 0.f) || score_scale == __builtin_huge_valf()) return XATTN_EINVAL;
-  const size_t need = xattn_score_workspace_size(B, Hq, M, stride, block);
-  if (workspace_bytes < need) return XATTN_EINVAL;
-  const int rp = M / stride;
-  if ((rp + 127) / 128 > (1 << 30)) return XATTN_EUNSUPPORTED;
-  float* part = static_cast<float*>(workspace);
-  float* lse_ws = part + (size_t)B * Hq * rp * (M / block);
-  auto q = static_cast<const bf16*>(Q);
-  auto k = static_cast<const bf16*>(K);
-  cudaStream_t st = as_stream(stream);
-  const int diag = pattern == XATTN_PATTERN_DIAGONAL ? 1 : 0;
-  if (C == 64)
-    return launch_score_c<64>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, diag, score_scale,
-                              scores, part, lse_ws, st);
-  return launch_score_c<128>(stride, q, k, B, Hq, Hkv, M, causal ? 1 : 0, diag, score_scale,
-                             scores, part, lse_ws, st);
 }
 
 int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C, int stride,
@@ -290,6 +301,56 @@ int xattn_select_ex(const float* scores, const float* param, int rule, int B, in
                     int32_t* nnz, void* workspace, size_t workspace_bytes, void* stream) {
   return select_common(scores, param, rule, B, Hq, nb, causal, row_ptr, col_idx, col_capacity,
                        nnz, workspace, workspace_bytes, stream);
+}
+
+size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block) {
+  const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block);
+  if (a == 0 && !(B == 0 || Hq == 0 || M == 0)) return 0;
+  const size_t a_al = (a + 255) & ~(size_t)255;
+  return a_al + xattn_select_workspace_size(B, Hq, block > 0 ? M / block : 0);
+}
+
+int xattn_score_select(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
+                       int stride, int block, int causal, float score_scale, const float* param,
+                       int rule, float* scores, int32_t* row_ptr, int32_t* col_idx,
+                       size_t col_capacity, int32_t* nnz, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, Hq, Hkv, M, C, block);
+  if (rc != XATTN_OK) return rc;
+  if (rule != kSelThreshold && rule != kSelTopK && rule != kSelRatio) return XATTN_EINVAL;
+  const int nb = M / block;
+  const long long rows = (long long)B * Hq * nb;
+  if (nb > kSelMaxNb) return XATTN_EUNSUPPORTED;
+  const long long worst = causal ? rows * (nb + 1) / 2 : rows * nb;
+  if (worst >= (1LL << 31) || rows >= (1LL << 31) - 1) return XATTN_EUNSUPPORTED;
+  if (!row_ptr || !nnz) return XATTN_EINVAL;
+  if (rows > 0 && (!param || !col_idx)) return XATTN_EINVAL;
+  if (workspace_bytes < xattn_score_select_workspace_size(B, Hq, M, stride, block))
+    return XATTN_EINVAL;
+  cudaStream_t st = as_stream(stream);
+  if (rows == 0) {
+    if (cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    return XATTN_OK;
+  }
+  if (!workspace || ((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
+  const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block);
+  const size_t a_al = (a + 255) & ~(size_t)255;
+  SelCut* cuts = reinterpret_cast<SelCut*>(static_cast<uint8_t*>(workspace) + a_al);
+  FusedSelect fs;
+  fs.param = param;
+  fs.rule = rule;
+  fs.cuts = cuts;
+  rc = score_common<true>(Q, K, B, Hq, Hkv, M, C, stride, block, causal,
+                          XATTN_PATTERN_ANTIDIAGONAL, score_scale, scores, workspace, a, stream,
+                          fs);
+  if (rc != XATTN_OK) return rc;
+  const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
+  select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
+                                                              row_ptr, col_idx);
+  return launch_status();
 }
 
 // ---- selection without a caller workspace -------------------------------

@@ -187,6 +187,28 @@ XATTN_API int xattn_select_ex(const float* scores, const float* param, int rule,
                               size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace bytes xattn_score_select needs: the scoring workspace (rounded up
+ * to 256 bytes) followed by the selection workspace.
+ */
+XATTN_API size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block);
+
+/*
+ * xattn_score_select - xattn_score followed by xattn_select_ex, fused
+ * [DuSA-Q2, XA-abs, XA-app, FP-RQ3]. The scoring kernel ranks and cuts every
+ * query-block row right after writing its scores, while the row is still in L2,
+ * so the selection needs only its scan and fill passes: three launches instead
+ * of four, and no second read of the score matrix. scores and the CSR
+ * (row_ptr, col_idx, nnz) are bit-identical to those of xattn_score with the
+ * antidiagonal pattern followed by xattn_select_ex with the same rule and param;
+ * every argument, layout and error has the meaning it has there.
+ */
+XATTN_API int xattn_score_select(const void* Q, const void* K, int B, int Hq, int Hkv, int M,
+                                 int C, int stride, int block, int causal, float score_scale,
+                                 const float* param, int rule, float* scores, int32_t* row_ptr,
+                                 int32_t* col_idx, size_t col_capacity, int32_t* nnz,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Largest number of selection rows (B*Hq*nb) that xattn_select_noalloc takes.
  */
 #define XATTN_SELECT_NOALLOC_MAX_ROWS 262144

@@ -181,3 +181,20 @@ def test_selftest_rejects_bad_limits():
     for bad in (0, -5, 2_000_000_000):
         assert xa._lib.xattn_selftest_wait_timeout(bad, FAKE, None) == xa.XATTN_EINVAL
     assert xa._lib.xattn_selftest_wait_timeout(1000, None, None) == xa.XATTN_EINVAL
+
+
+def test_fused_score_select_rejects_on_host():
+    assert xa.xattn_score_select_workspace_size(1, 2, 1024, 8) == \
+        ((xa.xattn_score_workspace_size(1, 2, 1024, 8) + 255) // 256 * 256 +
+         xa.xattn_select_workspace_size(1, 2, 8))
+    args = [FAKE, FAKE, 1, 4, 2, 1024, 128, 8, 128, 1, 0.03, FAKE, 0, FAKE, FAKE, FAKE, 1 << 20,
+            FAKE, FAKE, 1 << 40, None]
+    bad_rule = list(args)
+    bad_rule[12] = 7
+    assert xa._lib.xattn_score_select(*bad_rule) == xa.XATTN_EINVAL
+    small_ws = list(args)
+    small_ws[19] = 64
+    assert xa._lib.xattn_score_select(*small_ws) == xa.XATTN_EINVAL
+    bad_shape = list(args)
+    bad_shape[5] = 1000
+    assert xa._lib.xattn_score_select(*bad_shape) == xa.XATTN_EINVAL

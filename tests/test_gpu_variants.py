@@ -105,3 +105,46 @@ def test_threshold_rule_equals_select():
     assert a[2] == n
     np.testing.assert_array_equal(a[0], row_ptr.cpu().numpy())
     np.testing.assert_array_equal(a[1][:n], col.cpu().numpy()[:n])
+
+
+@pytest.mark.parametrize("M,C,Hq,Hkv,S,causal,B", [
+    (2048, 64, 1, 1, 8, True, 1),
+    (1152, 128, 4, 2, 8, True, 2),      # ragged score tile, two batch elements
+    (1024, 128, 2, 1, 4, False, 1),
+    (4096, 128, 4, 2, 16, True, 1),
+])
+def test_fused_score_select_equals_two_calls(M, C, Hq, Hkv, S, causal, B):
+    w = small_workload(M, C, Hq, Hkv, S, causal).with_(B=B)
+    _, (Q, K, _) = device_inputs(w)
+    nb = M // 128
+    sig = orc.default_score_scale(S, C)
+    rules = ((xa.XATTN_SELECT_THRESHOLD, [0.9, 0.7, 0.95, 0.6][:Hq]),
+             (xa.XATTN_SELECT_TOPK, [3.0, 1.0, 5.0, 2.0][:Hq]),
+             (xa.XATTN_SELECT_RATIO, [0.25, 0.5, 0.1, 1.0][:Hq]))
+    cap = xa.max_kept(B, Hq, nb, causal)
+    for rule, prm in rules:
+        param = torch.tensor(prm, dtype=torch.float32, device="cuda")
+        # reference: the two separate calls
+        sc1 = torch.empty((B, Hq, nb, nb), device="cuda")
+        ws1 = torch.empty(xa.xattn_score_workspace_size(B, Hq, M, S), dtype=torch.uint8,
+                          device="cuda")
+        xa.xattn_score(Q, K, S, causal, sig, sc1, ws1)
+        rp1 = torch.empty(B * Hq * nb + 1, dtype=torch.int32, device="cuda")
+        ci1 = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        nz1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        wss = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8,
+                          device="cuda")
+        xa.xattn_select_ex(sc1, param, rule, causal, rp1, ci1, nz1, wss)
+        # fused
+        sc2 = torch.empty_like(sc1)
+        rp2 = torch.empty_like(rp1)
+        ci2 = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+        nz2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ws2 = torch.empty(xa.xattn_score_select_workspace_size(B, Hq, M, S), dtype=torch.uint8,
+                          device="cuda")
+        xa.xattn_score_select(Q, K, param, rule, S, causal, sig, sc2, rp2, ci2, nz2, ws2)
+        torch.cuda.synchronize()
+        n = int(nz1.item())
+        assert torch.equal(sc1, sc2)
+        assert int(nz2.item()) == n and torch.equal(rp1, rp2)
+        assert torch.equal(ci1[:n], ci2[:n])
