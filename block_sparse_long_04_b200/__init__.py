@@ -46,6 +46,7 @@ SIGNATURES = {
     "xattn_score_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _Z, _P]),
     "xattn_select_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
     "xattn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _P, _P]),
+    "xattn_selftest_exp2": (_I, [_P, _P, ctypes.c_longlong, _P]),
     "xattn_score_select_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "xattn_score_select": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _Z,
                                 _P, _P, _Z, _P]),
@@ -242,6 +243,15 @@ def xattn_selftest_wait_timeout(limit_ns: int, timed_out, stream=None) -> None:
     _dev(timed_out)
     _check(_lib.xattn_selftest_wait_timeout(int(limit_ns), _ptr(timed_out), _stream(stream)),
            "xattn_selftest_wait_timeout")
+
+
+def xattn_selftest_exp2(x, y, stream=None) -> None:
+    """y = 2^x through the FMA-pipe exponential of the attention softmax."""
+    _dev(x, y)
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise ValueError("x and y must be float32 tensors of the same size")
+    _check(_lib.xattn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "xattn_selftest_exp2")
 
 
 def xattn_get_device_error(stream=None) -> int:

@@ -8,14 +8,18 @@
 //   warp 0, one lane  TMA producer: Q once, then the K and V tiles of the kept
 //                     blocks (in list order) into two rings of kStages stages with
 //                     their own full/empty barriers; K runs one block ahead of V.
-//   warp 1, one lane  S issuer and TMEM owner: S = Q K^T into TMEM (128 lanes x
-//                     128 fp32 columns); S of block j+1 is issued as soon as the
-//                     softmax has read S of block j.
-//   warp 2, one lane  PV issuer: per key half g (keys 64g..64g+63), O_g += P_g V_g
-//                     into its own TMEM accumulator. Issuing is split over two
+//   warp 1, one lane  S issuer and TMEM owner: S = Q K^T into one of two TMEM
+//                     buffers (128 lanes x 128 fp32 columns each); S of block j
+//                     goes to buffer j%2 as soon as the PV MMAs of block j-2,
+//                     which read P from that buffer, have completed, so the next
+//                     block's S is computed while the softmax works on this one.
+//   warps 2, 3,       PV issuers, one per key half g (keys 64g..64g+63):
+//   one lane each     O_g += P_g V_g into the half's own TMEM accumulator, as soon
+//                     as that half's P is written. Issuing is split over three
 //                     threads on different sub-partitions because one thread
 //                     cannot issue the 16 MMAs of a block and poll their barriers
-//                     as fast as the tensor core retires them; each issuer's
+//                     as fast as the tensor core retires them, and so that one
+//                     half's PV never queues behind the other's; each issuer's
 //                     commits track exactly its own MMAs.
 //   warps 4-11        softmax, two threads per query row (TMEM lane = row): warps
 //                     4-7 own keys 0-63 of every block, warps 8-11 keys 64-127.
@@ -28,8 +32,10 @@
 //                     Per block: read the half row of S, causal mask on the
 //                     diagonal block, fp32 base-2 softmax with the scale folded into
 //                     one FMA, lazy rescaling (O_g and l_g are rescaled only when
-//                     m_g grows by more than 2^8), P_g as bf16 into TMEM, where the
-//                     PV MMA reads it as its A operand.
+//                     m_g grows by more than 2^8), P_g as bf16 over the first 32
+//                     columns of its own half of the S buffer, where the PV MMA
+//                     reads it as its A operand. Only a rescale waits for the
+//                     previous block's PV.
 // Every role walks the row's list with the next entry's load already in flight
 // (ListIter), so no role waits on a global load inside its loop.
 // Every wait is bounded (sm100::mbar_wait); on a timeout the CTA raises
@@ -42,6 +48,10 @@
 namespace xattn {
 
 constexpr int kAttnTcThreads = 384;
+#ifndef XATTN_EXP2_EMU_PER4
+#define XATTN_EXP2_EMU_PER4 2
+#endif
+constexpr int kEmuPer4 = XATTN_EXP2_EMU_PER4;   // softmax pairs (of 4) on the FMA pipe
 
 template <int C>
 struct AttnTc {
@@ -55,10 +65,11 @@ struct AttnTc {
   static constexpr int kOffBar = kOffV + kStages * kTile;
   static constexpr int kOffX = kOffBar + 256;             // end-of-row (m, l) exchange
   static constexpr int kSmem = kOffX + 2 * 128 * 8 + 1024;  // + alignment slack
-  static constexpr int kTmemCols = 512;                   // S, O_0, O_1, P_0, P_1
-  static constexpr int kColS = 0;                         // 128 fp32 columns
-  static constexpr int kColO = 128;                       // + g * 128: C fp32 columns each
-  static constexpr int kColP = 384;                       // + g * 32: 64 bf16 keys each
+  static constexpr int kTmemCols = 512;                   // S_0, S_1, O_0, O_1
+  static constexpr int kColS = 0;                         // + b * 128: 128 fp32 columns each
+  static constexpr int kColO = 256;                       // + g * 128: C fp32 columns each
+  // P_g of the block in S buffer b: 64 bf16 keys packed into the first 32
+  // columns of that buffer's half g (kColS + b * 128 + g * 64)
 };
 
 // Walks the kept-block list of one row, skipping entries outside [0, nb) and,
@@ -108,15 +119,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* k_full = bars;            // [ST] K tile of a block landed
   uint64_t* k_empty = bars + ST;      // [ST] its S MMA completed
   uint64_t* v_full = bars + 2 * ST;   // [ST] V tile of a block landed
-  uint64_t* v_empty = bars + 3 * ST;  // [ST] both of its PV MMAs completed
+  uint64_t* v_empty = bars + 3 * ST;  // [ST] both of its PV MMAs completed (2 issuers)
   uint64_t* q_full = bars + 4 * ST;
-  uint64_t* s_full = q_full + 1;      // S of the current block computed
-  uint64_t* s_free = q_full + 2;      // all 8 softmax warps have read it
-  uint64_t* p_full = q_full + 3;      // [2] P_g written (4 warps each)
-  uint64_t* o_done = q_full + 5;      // [2] PV_g of the block completed
-  uint64_t* drain = q_full + 7;       // [2] S issuer, PV issuer
-  uint64_t* x_full = q_full + 9;      // end-of-row (m_g, l_g) published (8 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 10);
+  uint64_t* s_full = q_full + 1;      // [2 buffers] S of the block computed
+  uint64_t* s_free = q_full + 3;      // [2 buffers] both PV MMAs reading P from it completed (2)
+  uint64_t* p_full = q_full + 5;      // [2 halves][2 buffers] P_g written (4 warps each)
+  uint64_t* o_done = q_full + 9;      // [2 halves] PV_g of the block completed
+  uint64_t* drain = q_full + 11;      // [3] S issuer, PV issuers of halves 0 and 1
+  uint64_t* x_full = q_full + 14;     // end-of-row (m_g, l_g) published (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* xchg = reinterpret_cast<float2*>(smem + L::kOffX);   // [2 half][128]
 
@@ -133,14 +144,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (tid == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 2);
     }
     mbar_init(q_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
-    mbar_init(&p_full[0], 4); mbar_init(&p_full[1], 4);
-    mbar_init(&o_done[0], 1); mbar_init(&o_done[1], 1);
-    mbar_init(&drain[0], 1); mbar_init(&drain[1], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 2);
+      mbar_init(&p_full[2 * i], 4); mbar_init(&p_full[2 * i + 1], 4);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(&drain[0], 1); mbar_init(&drain[1], 1); mbar_init(&drain[2], 1);
     mbar_init(x_full, 8);
     *abort_flag = 0;
     fence_mbar_init();
@@ -158,7 +170,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem + L::kColS;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -207,7 +218,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int jj = (nv > ST ? nv - ST : 0); jj < nv; ++jj)
         mbar_wait(&v_full[jj % ST], (jj / ST) & 1, &no_abort);
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp >= 1 && warp <= 3) {
     // ------------------------------------------------- S and PV issuers
     if (lane == 0) {
       // descriptors built once; per MMA only the start address (16-byte units,
@@ -226,43 +237,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         auto issue_S = [&](int j) {
           const int st = j % ST;
           const uint64_t dKs = dK + (uint64_t)((st * L::kTile) >> 4);
+          const uint32_t tSb = tmem + L::kColS + (j & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * L::kRegion + (kk & 3) * 32) >> 4;
-            mma_f16_ss(tS, dQ + off, dKs + off, idS, kk > 0);
+            mma_f16_ss(tSb, dQ + off, dKs + off, idS, kk > 0);
           }
-          mma_commit(s_full);
+          mma_commit(&s_full[j & 1]);
           mma_commit(&k_empty[st]);
         };
-        ok = have_cur && mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
-        if (ok) {
-          tc_fence_after();
-          issue_S(0);
-        }
-        for (int j = 0; ok && have_nxt; ++j) {
-          ok = mbar_wait(&k_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag) &&
-               mbar_wait(s_free, j & 1, abort_flag);
+        ok = have_cur && mbar_wait(q_full, 0, abort_flag);
+        for (int j = 0; ok && have_cur; ++j) {
+          // buffer j%2 is free once the PV MMAs of block j-2 have read its P
+          ok = mbar_wait(&k_full[j % ST], (j / ST) & 1, abort_flag) &&
+               (j < 2 || mbar_wait(&s_free[j & 1], ((j >> 1) - 1) & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
-          issue_S(j + 1);
-          have_nxt = li.next() >= 0;
+          issue_S(j);
+          have_cur = have_nxt;
+          have_nxt = have_cur && li.next() >= 0;
         }
       } else {
+        const int g = warp - 2;              // key half of this PV issuer
         for (int j = 0; ok && have_cur; ++j) {
           const int st = j % ST;
-          if (!(ok = mbar_wait(&v_full[st], (j / ST) & 1, abort_flag))) break;
-          for (int g = 0; g < 2; ++g) {
-            if (!(ok = mbar_wait(&p_full[g], j & 1, abort_flag))) break;
-            tc_fence_after();
-            const uint64_t dVg = dV + (uint64_t)((st * L::kTile + g * 4 * 2048) >> 4);
+          const int b = j & 1;
+          if (!(ok = mbar_wait(&v_full[st], (j / ST) & 1, abort_flag) &&
+                     mbar_wait(&p_full[2 * g + b], (j >> 1) & 1, abort_flag)))
+            break;
+          tc_fence_after();
+          const uint64_t dVg = dV + (uint64_t)((st * L::kTile + g * 4 * 2048) >> 4);
+          const uint32_t tP = tmem + L::kColS + b * 128 + g * 64;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)     // keys 64g + 16kk .. +15 (8 TMEM columns)
-              mma_f16_ts(tmem + L::kColO + g * 128, tmem + L::kColP + g * 32 + kk * 8,
-                         dVg + (kk * 2048 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&o_done[g]);
-          }
-          if (!ok) break;
+          for (int kk = 0; kk < 4; ++kk)     // keys 64g + 16kk .. +15 (8 TMEM columns)
+            mma_f16_ts(tmem + L::kColO + g * 128, tP + kk * 8, dVg + (kk * 2048 >> 4), idPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&o_done[g]);
           mma_commit(&v_empty[st]);
+          mma_commit(&s_free[b]);
           have_cur = have_nxt;
           have_nxt = have_cur && li.next() >= 0;
         }
@@ -277,9 +289,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int g = (warp >= 8) ? 1 : 0;                 // keys [64g, 64g + 64) of each block
     const int q_row = (warp & 3) * 32 + lane;          // row within the query block
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tSg = tS + lane_off + g * 64;
+    const uint32_t tSg = tmem + lane_off + L::kColS + g * 64;   // + b * 128
     const uint32_t tOg = tmem + lane_off + L::kColO + g * 128;
-    const uint32_t tPg = tmem + lane_off + L::kColP + g * 32;
     const int k0 = g * 64;
     float m = kNegInf, l = 0.f;
     int j = 0;
@@ -287,16 +298,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ListIter li;
     li.init(col_idx, beg, end, nb, r, causal != 0, DENSE);
     for (int c = li.next(); c >= 0; c = li.next()) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float s[64];
-      tmem_ld32(tSg, s);
-      tmem_ld32(tSg + 32, s + 32);
+      tmem_ld32(tSg + b * 128, s);
+      tmem_ld32(tSg + b * 128 + 32, s + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
 
       // half-row max of the raw logits (the scale is positive); masked keys of
       // the diagonal block are set to -inf first, on the diagonal block only
@@ -329,24 +338,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
       float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
+      // kEmuPer4 of every 4 pairs take the FMA-pipe exponential, the rest MUFU,
+      // so that neither unit alone sets the pace of the block
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
         const float2 x = ffma2(make_float2(s[i], s[i + 1]), sc2, nm2);
-        s[i] = ex2(x.x);
-        s[i + 1] = ex2(x.y);
+        if (((i >> 1) & 3) < kEmuPer4) {
+          const float2 e = ex2_poly2(x);
+          s[i] = e.x;
+          s[i + 1] = e.y;
+        } else {
+          s[i] = ex2(x.x);
+          s[i + 1] = ex2(x.y);
+        }
         ps[(i >> 1) & 3] = fadd2(ps[(i >> 1) & 3], make_float2(s[i], s[i + 1]));
       }
       const float2 pq = fadd2(fadd2(ps[0], ps[1]), fadd2(ps[2], ps[3]));
       const float rs = pq.x + pq.y;
       l = l * corr + rs;
 
-      // PV_g of the previous block must be complete: P_g free, O_g stable
-      if (j > 0) {
+      // a rescale needs O_g stable: PV_g of the previous block complete
+      if (__any_sync(0xffffffffu, resc)) {
         ok = __all_sync(0xffffffffu, mbar_wait(&o_done[g], (j - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
         for (int q = 0; q < C / 32; ++q) {
           float o[32];
@@ -358,18 +373,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         tmem_wait_st();
       }
-      // P_g half row -> TMEM (A operand of the PV MMA): 64 bf16 keys packed two
-      // per 32-bit column, one store per thread
+      // P_g half row -> TMEM over the S columns this thread has read (A operand
+      // of the PV MMA): 64 bf16 keys packed two per 32-bit column
       {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        tmem_st32(tPg, reinterpret_cast<const float*>(pk));
+        tmem_st32(tSg + b * 128, reinterpret_cast<const float*>(pk));
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[g]);
+      if (lane == 0) mbar_arrive(&p_full[2 * g + b]);
       ++j;
     }
 

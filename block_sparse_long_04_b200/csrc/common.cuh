@@ -93,6 +93,29 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return *reinterpret_cast<float2*>(&ud);
 }
 
+// 2^x for two lanes on the FMA and integer pipes instead of MUFU, for x <= 127
+// (-inf allowed). Range reduction: n = round-to-nearest(x) via the 1.5 * 2^23
+// addition, f = x - n in [-1/2, 1/2], both exact; 2^f = 1 + f(c1 + f(c2 + f c3)),
+// the cubic of least maximum relative error on [-1/2, 1/2] with constant term 1
+// (fit_exp2_poly.py, relative error 1.01e-4 in fp32); 2^n is added to the
+// exponent field as an integer. x is clamped to -127 first, where that sum is
+// the bit pattern of +0, so -inf and every x <= -127 give exactly 0.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  constexpr float c1 = 0.6932829022407532f, c2 = 0.2422109693288803f,
+                  c3 = 0.055009059607982635f;
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(1.f, 1.f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Byte offset of 16-byte chunk `ch` of row `row` in a tile whose rows are
 // `row_bytes` long, XOR-swizzled on the low three chunk bits so that eight
 // consecutive rows at the same logical chunk hit eight different bank groups.

@@ -2,6 +2,8 @@
 // The contract of every entry point is documented in include/xattn.h.
 #include "xattn.h"
 
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -35,6 +37,20 @@ int ensure_smem_limit(F* kern, int bytes, unsigned long long* done_mask) {
 
 inline int launch_status() {
   return cudaGetLastError() == cudaSuccess ? XATTN_OK : XATTN_ECUDA;
+}
+
+// y = 2^x through ex2_poly2, two elements per thread (grid-stride)
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                     long long n) {
+  const long long pairs = (n + 1) / 2;
+  for (long long p = blockIdx.x * (long long)blockDim.x + threadIdx.x; p < pairs;
+       p += (long long)gridDim.x * blockDim.x) {
+    const long long i = 2 * p;
+    const bool two = i + 1 < n;
+    const float2 e = ex2_poly2(make_float2(x[i], two ? x[i + 1] : 0.f));
+    y[i] = e.x;
+    if (two) y[i + 1] = e.y;
+  }
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
@@ -426,6 +442,15 @@ int xattn_selftest_wait_timeout(long long limit_ns, int32_t* timed_out, void* st
   if (limit_ns < 1 || limit_ns > 1000000000LL || timed_out == nullptr) return XATTN_EINVAL;
   sm100::wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(
       (unsigned long long)limit_ns, timed_out);
+  return launch_status();
+}
+
+int xattn_selftest_exp2(const float* x, float* y, long long n, void* stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return XATTN_EINVAL;
+  if (n == 0) return XATTN_OK;
+  const long long pairs = (n + 1) / 2;
+  const unsigned grid = (unsigned)std::min<long long>((pairs + 255) / 256, 148LL * 16);
+  exp2_selftest_kernel<<<grid, 256, 0, as_stream(stream)>>>(x, y, n);
   return launch_status();
 }
 

@@ -282,6 +282,17 @@ XATTN_API int xattn_dense_attn(const void* Q, const void* K, const void* V,
 XATTN_API int xattn_selftest_wait_timeout(long long limit_ns, int32_t* timed_out, void* stream);
 
 /*
+ * xattn_selftest_exp2 - diagnostic of the FMA-pipe base-2 exponential that the
+ * attention softmax uses for part of its elements instead of the hardware
+ * approximation (the pages have no counterpart). y[i] = 2^x[i] for n fp32
+ * values (device arrays, n >= 0): relative error at most 1.1e-4 for x in
+ * [-126, 127]; exactly 0 for x <= -127 and for -inf; a value in [0, 2^-126]
+ * in between. Larger x are outside its domain. Returns XATTN_EINVAL for n < 0
+ * or a null array with n > 0.
+ */
+XATTN_API int xattn_selftest_exp2(const float* x, float* y, long long n, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's error
  * word (XATTN_OK if no device-side condition was raised since the last call).
  * Returns XATTN_ECUDA if the synchronisation itself failed.

@@ -198,3 +198,9 @@ def test_fused_score_select_rejects_on_host():
     bad_shape = list(args)
     bad_shape[5] = 1000
     assert xa._lib.xattn_score_select(*bad_shape) == xa.XATTN_EINVAL
+
+
+def test_exp2_selftest_rejects_on_host():
+    assert xa._lib.xattn_selftest_exp2(FAKE, FAKE, -1, None) == xa.XATTN_EINVAL
+    assert xa._lib.xattn_selftest_exp2(None, FAKE, 4, None) == xa.XATTN_EINVAL
+    assert xa._lib.xattn_selftest_exp2(None, None, 0, None) == xa.XATTN_OK

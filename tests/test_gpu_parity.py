@@ -154,6 +154,8 @@ ATTN_CASES = [
     (1536, 128, 2, 1, False),
     (128, 64, 2, 2, True),
     (2048, 128, 8, 8, False),
+    (1152, 128, 2, 1, True),     # odd block count: the last query block has no partner
+    (1408, 64, 2, 2, False),
 ]
 
 
@@ -212,6 +214,45 @@ def test_attention_skips_invalid_entries_and_empty_rows():
     o, l = orc.block_sparse_attention(q, k, v, kept, 128, True, 0.125, rows=[1, 2, 3])
     P.assert_outputs_close(got[128:], o)
     np.testing.assert_allclose(gl[128:], l, rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_sparse_attention_list_order_does_not_matter(causal):
+    """Kept lists in descending or shuffled order: every entry of each row is
+    still attended exactly once (the two query blocks of a CTA merge their lists
+    step by step, which must not depend on the lists being ascending)."""
+    M, C, Hq, Hkv = 1280, 128, 2, 1
+    w = small_workload(M, C, Hq, Hkv, 8, causal)
+    (Qb, Kb, Vb), (Q, K, V) = device_inputs(w)
+    nb = M // 128
+    rng = np.random.default_rng(11)
+    kept = {}
+    for h in range(Hq):
+        for r in range(nb):
+            n = r + 1 if causal else nb
+            pick = sorted(set(rng.choice(n, size=max(1, n // 2), replace=False).tolist()) | {r})
+            kept.setdefault((0, h), {})[r] = pick
+    rows, ptr = [], [0]
+    for h in range(Hq):
+        for r in range(nb):
+            lst = list(kept[(0, h)][r])
+            mode = (r + h) % 3
+            if mode == 1:
+                lst = lst[::-1]
+            elif mode == 2:
+                lst = rng.permutation(lst).tolist()
+            rows.extend(lst)
+            ptr.append(len(rows))
+    rp = torch.tensor(ptr, dtype=torch.int32, device="cuda")
+    ci = torch.tensor(rows, dtype=torch.int32, device="cuda")
+    O = torch.empty_like(Q)
+    xa.xattn_sparse_attn(Q, K, V, rp, ci, causal, 1 / math.sqrt(C), O)
+    got = bf16_to_np(O)
+    grp = Hq // Hkv
+    for h in range(Hq):
+        q, k, v = (orc.bf16_to_f64(x) for x in (Qb[0, h], Kb[0, h // grp], Vb[0, h // grp]))
+        o, _ = orc.block_sparse_attention(q, k, v, kept[(0, h)], 128, causal, 1 / math.sqrt(C))
+        P.assert_outputs_close(got[0, h], o, f"O head {h}")
 
 
 def _pipeline(w, Q, K, V, tau, with_lse=False):
