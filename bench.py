@@ -63,7 +63,8 @@ def workload_of(a):
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_llama8b_gqa_128k.json")
-KERNEL_SOURCES = {"attn_tc": ["attn_tc.cuh"], "score_tc": ["score_tc.cuh"]}
+KERNEL_SOURCES = {"attn_tc": ["attn_tc.cuh", "common.cuh", "sm100.cuh"],
+                  "score_tc": ["score_tc.cuh", "select.cuh", "common.cuh", "sm100.cuh"]}
 
 
 def kernel_source_hash(kernel: str) -> str:
