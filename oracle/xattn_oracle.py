@@ -39,6 +39,8 @@ Readings where the pages are silent (each is exercised by the pins in tests/):
 - ties: descending score, then ascending block index.
 - the diagonal block is added after thresholding if it is not already kept.
 - GQA: query head h scores against KV head h // (Hq/Hkv), with its own tau_h.
+- GQA-shared selection (a variant the pages do not define, used only when asked
+  for): the query heads of one KV group share the union of their own kept lists.
 - sparse attention scale 1/sqrt(C); causal mask j <= i at token granularity.
 
 Parity pins for every function live in tests/test_oracle_pins.py; none of them
@@ -53,7 +55,7 @@ __all__ = [
     "block_scores", "select_row", "select_row_topk", "select_row_ratio", "ratio_count",
     "select_blocks", "selection_margins", "to_csr",
     "block_sparse_attention", "dense_attention", "layer_block_scores",
-    "layer_select", "layer_sparse_attention",
+    "layer_select", "layer_sparse_attention", "select_group_union", "layer_select_group",
 ]
 
 
@@ -309,4 +311,35 @@ def layer_sparse_attention(Qb, Kb, Vb, Hkv: int, kept_by_head, block: int, causa
         k = bf16_to_f64(Kb[b, h // grp])
         v = bf16_to_f64(Vb[b, h // grp])
         out[(b, h)] = block_sparse_attention(q, k, v, kept, block, causal, scale, rows)
+    return out
+
+
+def select_group_union(member_kept):
+    """Kept lists shared by the query heads of one KV group: per query block, the
+    union of the members' own kept lists.
+
+    Not the pages' definition (there each head keeps its own minimal set, XAttention
+    summary, "Approach"); a variant for GQA models in which one K/V block list serves
+    every query head of the group. Each member's own set is contained in the union,
+    so each member still covers at least its own threshold mass.
+    member_kept: list over the group's heads of {r: kept}. Returns {r: ascending}.
+    """
+    out = {}
+    for r in member_kept[0]:
+        u = set()
+        for kept in member_kept:
+            u.update(int(c) for c in kept[r])
+        out[r] = np.array(sorted(u), dtype=np.int64)
+    return out
+
+
+def layer_select_group(kept_by_head, Hq: int, Hkv: int):
+    """{(b, kvh): {r: union}} from {(b, h): {r: kept}}; head h belongs to KV head
+    h // (Hq/Hkv)."""
+    grp = Hq // Hkv
+    out = {}
+    for b in sorted({b for (b, _) in kept_by_head}):
+        for kvh in range(Hkv):
+            out[(b, kvh)] = select_group_union(
+                [kept_by_head[(b, h)] for h in range(kvh * grp, (kvh + 1) * grp)])
     return out

@@ -372,3 +372,45 @@ def test_planted_wrong_tie_break_is_caught(monkeypatch):
     with pytest.raises(AssertionError):
         for seed in range(40):
             test_selection_is_a_minimal_set(seed)
+
+
+def test_group_union_hand_example_and_threshold_mass():
+    """GQA-shared selection: a hand-worked union, and every member head still
+    covers its own threshold mass over the shared list (checked on the scores,
+    independently of how the union is formed)."""
+    got = orc.select_group_union([{0: np.array([0]), 3: np.array([0, 3])},
+                                  {0: np.array([0]), 3: np.array([1, 3])},
+                                  {0: np.array([0]), 3: np.array([3])}])
+    assert got[0].tolist() == [0] and got[3].tolist() == [0, 1, 3]
+    rng = np.random.default_rng(5)
+    nb, G = 9, 4
+    for causal in (True, False):
+        scores = [rng.gamma(0.4, size=(nb, nb)) for _ in range(G)]
+        if causal:
+            scores = [np.tril(x) for x in scores]
+        scores = [x / x.sum(axis=1, keepdims=True) for x in scores]
+        taus = [0.5, 0.7, 0.9, 0.95]
+        kept = [orc.select_blocks(scores[i], taus[i], causal) for i in range(G)]
+        union = orc.select_group_union(kept)
+        for r in range(nb):
+            u = union[r].tolist()
+            assert u == sorted(set(u)) and r in u
+            assert all(0 <= c <= (r if causal else nb - 1) for c in u)
+            for i in range(G):
+                assert scores[i][r, u].sum() >= taus[i] - 1e-12
+                assert set(kept[i][r].tolist()) <= set(u)
+            # no block that no member kept
+            assert set(u) <= set().union(*(set(kept[i][r].tolist()) for i in range(G)))
+        # a group of one is the head's own selection
+        solo = orc.select_group_union([kept[0]])
+        assert all(solo[r].tolist() == kept[0][r].tolist() for r in range(nb))
+
+
+def test_layer_group_maps_heads_to_their_kv_head():
+    kept = {(0, h): {0: np.array([0]), 1: np.array([h % 2, 1])} for h in range(4)}
+    g = orc.layer_select_group(kept, Hq=4, Hkv=2)
+    assert sorted(g) == [(0, 0), (0, 1)]
+    assert g[(0, 0)][1].tolist() == [0, 1] and g[(0, 1)][1].tolist() == [0, 1]
+    kept[(0, 2)][1] = np.array([1])
+    kept[(0, 3)][1] = np.array([1])
+    assert orc.layer_select_group(kept, Hq=4, Hkv=2)[(0, 1)][1].tolist() == [1]
