@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fused-select", action="store_true",
                     help="score and select in the one fused call instead of two calls")
+    ap.add_argument("--group-select", action="store_true",
+                    help="GQA-shared kept lists (union over each KV group; a variant the "
+                         "method does not define) instead of per-head lists")
     return ap.parse_args()
 
 
@@ -274,9 +277,30 @@ def main():
     ss = xa.default_score_scale(w.stride, w.C)
     sa = 1 / math.sqrt(w.C)
 
+    G = w.Hq // w.Hkv
+    if a.group_select:
+        g_rp = torch.empty(w.B * w.Hkv * w.nb + 1, dtype=torch.int32, device=dev)
+        g_col = torch.empty(xa.max_kept(w.B, w.Hkv, w.nb, w.causal), dtype=torch.int32,
+                            device=dev)
+        g_ws = torch.empty(xa.xattn_select_group_workspace_size(w.B, w.Hq, w.Hkv, w.nb),
+                           dtype=torch.uint8, device=dev)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
+        if a.group_select:
+            xa.xattn_score(Q, K, w.stride, w.causal, ss, bufs.scores, bufs.score_ws,
+                           stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            xa.xattn_select_group(bufs.scores, tau, xa.XATTN_SELECT_THRESHOLD, w.Hkv, w.causal,
+                                  g_rp, g_col, bufs.nnz, g_ws, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+            xa.xattn_sparse_attn_group(Q, K, V, g_rp, g_col, w.causal, sa, bufs.O, stream=stream)
+            if ev is not None:
+                ev[3].record(stream)
+            return
         if not a.fused_select:
             xa.xattn_score(Q, K, w.stride, w.causal, ss, bufs.scores, bufs.score_ws,
                            stream=stream)
@@ -300,7 +324,8 @@ def main():
 
     # unfused: score 1, select 3 (count, scan, fill), attention 1;
     # fused: score with row cuts 1, scan 1, fill 1, attention 1
-    launches_per_step = 4 if a.fused_select else 5
+    # grouped: score 1, select 4 (count, group count, scan, group fill), attention 1
+    launches_per_step = 6 if a.group_select else (4 if a.fused_select else 5)
     for _ in range(a.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -325,7 +350,7 @@ def main():
     st_select = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     st_attn = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
 
-    nnz = int(bufs.nnz.item())
+    nnz = int(bufs.nnz.item()) * (G if a.group_select else 1)   # attended (head, block) pairs
     if xa.xattn_get_device_error() != xa.XATTN_OK:
         raise RuntimeError("device error during the timed steps")
     b2, C = w.block ** 2, w.C
@@ -339,7 +364,8 @@ def main():
                 "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": attn_tflops / pk["bf16_sustained"],
                 "peak_source": f"{pk['source']} bf16 sustained (kernel runs inside a long step)",
-                "traffic": measured_traffic("attn_tc", w.name, w.stride),
+                "traffic": (None if a.group_select
+                            else measured_traffic("attn_tc", w.name, w.stride)),
                 "algorithmic": "4*b^2*C FLOP per kept (head, query block, key block), "
                                "diagonal blocks counted in full"}
     score_flops = (1.0 if w.causal else 2.0) * w.M * w.M * C * w.Hq * w.B / w.stride
@@ -441,7 +467,10 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(w), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "config": dict(config_of(w), selection=(
+            "GQA-shared union over each KV group (variant)" if a.group_select else
+            "per head, fused with scoring" if a.fused_select else "per head")),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * a.steps, "clocks": clk.summary(), **extra,
     }
     if rank == 0:

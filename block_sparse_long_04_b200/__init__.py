@@ -47,6 +47,10 @@ SIGNATURES = {
     "xattn_select_ex": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
     "xattn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _P, _P]),
     "xattn_selftest_exp2": (_I, [_P, _P, ctypes.c_longlong, _P]),
+    "xattn_select_group_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "xattn_select_group": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
+    "xattn_sparse_attn_group": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
+                                     _P]),
     "xattn_score_select_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "xattn_score_select": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _Z,
                                 _P, _P, _Z, _P]),
@@ -167,6 +171,23 @@ def xattn_select_ex(scores, param, rule: int, causal: bool, row_ptr, col_idx, nn
     _check(rc, "xattn_select_ex")
 
 
+def xattn_select_group_workspace_size(B: int, Hq: int, Hkv: int, nb: int) -> int:
+    return int(_lib.xattn_select_group_workspace_size(B, Hq, Hkv, nb))
+
+
+def xattn_select_group(scores, param, rule: int, Hkv: int, causal: bool, row_ptr, col_idx, nnz,
+                       workspace, stream=None) -> None:
+    """GQA-shared kept lists (a variant): per (b, kv head, query block) the union of
+    the group's per-head selections; CSR over B*Hkv*nb rows."""
+    _dev(scores, param, row_ptr, col_idx, nnz, workspace)
+    B, Hq, nb, _ = scores.shape
+    rc = _lib.xattn_select_group(_ptr(scores), _ptr(param), int(rule), B, Hq, Hkv, nb,
+                                 int(causal), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                 _ptr(nnz), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "xattn_select_group")
+
+
 def xattn_score_select_workspace_size(B: int, Hq: int, M: int, stride: int, block: int = 128) -> int:
     return int(_lib.xattn_score_select_workspace_size(B, Hq, M, stride, block))
 
@@ -223,6 +244,19 @@ def xattn_sparse_attn(Q, K, V, row_ptr, col_idx, causal: bool, softmax_scale: fl
                                 Hkv, M, C, block, int(causal), float(softmax_scale), _ptr(O),
                                 _ptr(lse), _stream(stream))
     _check(rc, "xattn_sparse_attn")
+
+
+def xattn_sparse_attn_group(Q, K, V, row_ptr, col_idx, causal: bool, softmax_scale: float, O,
+                            lse=None, block: int = 128, stream=None) -> None:
+    """xattn_sparse_attn over GQA-shared lists (CSR rows per batch, KV head, query block)."""
+    _dev(Q, K, V, row_ptr, col_idx, O, lse)
+    _bf16(Q, K, V, O)
+    B, Hq, M, C = Q.shape
+    Hkv = K.shape[1]
+    rc = _lib.xattn_sparse_attn_group(_ptr(Q), _ptr(K), _ptr(V), _ptr(row_ptr), _ptr(col_idx), B,
+                                      Hq, Hkv, M, C, block, int(causal), float(softmax_scale),
+                                      _ptr(O), _ptr(lse), _stream(stream))
+    _check(rc, "xattn_sparse_attn_group")
 
 
 def xattn_dense_attn(Q, K, V, causal: bool, softmax_scale: float, O, lse=None, block: int = 128,

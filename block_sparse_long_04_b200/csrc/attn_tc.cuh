@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kAttnTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ row_ptr,
                const int32_t* __restrict__ col_idx, int Hq, int Hkv, int M, int causal,
-               float scale_log2, bf16* __restrict__ O, float* __restrict__ lse) {
+               int group_rows, float scale_log2, bf16* __restrict__ O, float* __restrict__ lse) {
   using L = AttnTc<C>;
   constexpr int ST = L::kStages;
   using namespace sm100;
@@ -131,7 +131,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int r = nb - 1 - (int)blockIdx.x;   // longest rows first
   const int bh = blockIdx.y;
   const int b = bh / Hq, h = bh % Hq, kvh = h / (Hq / Hkv);
-  const size_t row = (size_t)bh * nb + r;
+  // the kept list: per (batch, query head) row, or shared by the KV group
+  const size_t row = (size_t)(group_rows ? b * Hkv + kvh : bh) * nb + r;
   int beg, end;
   if (DENSE) { beg = 0; end = causal ? r + 1 : nb; }
   else { beg = row_ptr[row]; end = row_ptr[row + 1]; }

@@ -36,6 +36,8 @@ struct SelCut {
   int count;     // kept entries of the row, diagonal included
 };
 
+constexpr int kSelMaxGroup = 64;  // query heads per KV head for GQA-shared lists
+
 // a ranks before b: higher score first, equal scores by smaller index
 __device__ __forceinline__ bool ranks_before(float sa, int ia, float sb, int ib) {
   return sa > sb || (sa == sb && ia < ib);
@@ -159,6 +161,11 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   return cut;
 }
 
+// block c of row r is kept under the row's cut (the diagonal always is)
+__device__ __forceinline__ bool kept_by_cut(float s, int c, int r, const SelCut& cut) {
+  return c == r || ranks_before(s, c, cut.score, cut.index) || (s == cut.score && c == cut.index);
+}
+
 __global__ void __launch_bounds__(kSelThreads)
 select_count_kernel(const float* __restrict__ scores, const float* __restrict__ tau, int Hq, int nb,
                     int causal, SelCut* __restrict__ cuts, int rule) {
@@ -213,10 +220,7 @@ select_fill_kernel(const float* __restrict__ scores, const SelCut* __restrict__ 
   const float* srow = scores + (size_t)row * nb;
   const int per = (n + kSelThreads - 1) / kSelThreads;
   const int lo = threadIdx.x * per, hi = min(n, lo + per);
-  auto kept = [&](int c) {
-    const float s = srow[c];
-    return c == r || ranks_before(s, c, cut.score, cut.index) || (s == cut.score && c == cut.index);
-  };
+  auto kept = [&](int c) { return kept_by_cut(srow[c], c, r, cut); };
   int cnt = 0;
   for (int c = lo; c < hi; ++c) cnt += kept(c) ? 1 : 0;
   int total;
@@ -224,6 +228,69 @@ select_fill_kernel(const float* __restrict__ scores, const SelCut* __restrict__ 
   // the row's count bounds the writes even if cuts and scores disagree
   for (int c = lo; c < hi && pos < cut.count; ++c)
     if (kept(c)) col_idx[base + pos++] = c;
+}
+
+// ---- GQA-shared lists ------------------------------------------------------
+// Block c of query block r is kept for KV group (b, kvh) when any query head of
+// the group keeps it under its own cut. One CTA per group row
+// (b * Hkv + kvh) * nb + r; the G = Hq / Hkv member rows are
+// (b * Hq + kvh * G + i) * nb + r.
+struct GroupRow {
+  int r, n, G;
+  size_t row0;   // first member row
+  __device__ __forceinline__ GroupRow(int grow, int Hq, int Hkv, int nb, int causal) {
+    const int bk = grow / nb;
+    r = grow % nb;
+    n = causal ? r + 1 : nb;
+    G = Hq / Hkv;
+    row0 = ((size_t)(bk / Hkv) * Hq + (size_t)(bk % Hkv) * G) * nb + r;
+  }
+};
+
+__device__ __forceinline__ bool group_keeps(const float* __restrict__ scores, const SelCut* cut_s,
+                                            const GroupRow& g, int nb, int c) {
+  bool any = false;
+  for (int i = 0; i < g.G && !any; ++i)
+    any = kept_by_cut(scores[(g.row0 + (size_t)i * nb) * nb + c], c, g.r, cut_s[i]);
+  return any;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_group_count_kernel(const float* __restrict__ scores, const SelCut* __restrict__ cuts,
+                          int Hq, int Hkv, int nb, int causal, SelCut* __restrict__ gcuts) {
+  __shared__ int red[32];
+  __shared__ SelCut cut_s[kSelMaxGroup];
+  const GroupRow g((int)blockIdx.x, Hq, Hkv, nb, causal);
+  for (int i = threadIdx.x; i < g.G; i += kSelThreads) cut_s[i] = cuts[g.row0 + (size_t)i * nb];
+  __syncthreads();
+  int cnt = 0;
+  for (int c = threadIdx.x; c < g.n; c += kSelThreads) cnt += group_keeps(scores, cut_s, g, nb, c);
+  int total;
+  block_exclusive_scan_i32(cnt, red, total);
+  if (threadIdx.x == 0) gcuts[blockIdx.x] = SelCut{0.f, 0, total};
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_group_fill_kernel(const float* __restrict__ scores, const SelCut* __restrict__ cuts,
+                         const SelCut* __restrict__ gcuts, int Hq, int Hkv, int nb, int causal,
+                         const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx) {
+  __shared__ int red[32];
+  __shared__ SelCut cut_s[kSelMaxGroup];
+  const int grow = blockIdx.x;
+  const GroupRow g(grow, Hq, Hkv, nb, causal);
+  const int base = row_ptr[grow];
+  const int count = gcuts[grow].count;
+  if (row_ptr[grow + 1] - base != count) return;   // lists withdrawn (capacity)
+  for (int i = threadIdx.x; i < g.G; i += kSelThreads) cut_s[i] = cuts[g.row0 + (size_t)i * nb];
+  __syncthreads();
+  const int per = (g.n + kSelThreads - 1) / kSelThreads;
+  const int lo = threadIdx.x * per, hi = min(g.n, lo + per);
+  int cnt = 0;
+  for (int c = lo; c < hi; ++c) cnt += group_keeps(scores, cut_s, g, nb, c);
+  int total;
+  int pos = block_exclusive_scan_i32(cnt, red, total);
+  for (int c = lo; c < hi && pos < count; ++c)
+    if (group_keeps(scores, cut_s, g, nb, c)) col_idx[base + pos++] = c;
 }
 
 }  // namespace xattn

@@ -148,8 +148,8 @@ int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int 
 
 template <int C, bool DENSE>
 int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
-                   const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal, float scale,
-                   bf16* O, float* lse, cudaStream_t st) {
+                   const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal,
+                   int group_rows, float scale, bf16* O, float* lse, cudaStream_t st) {
   auto kern = attn_tc_kernel<C, DENSE>;
   constexpr int smem = AttnTc<C>::kSmem;
   static unsigned long long done = 0;
@@ -161,14 +161,15 @@ int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* r
     return XATTN_ECUDA;
   dim3 grid(M / 128, B * Hq);
   kern<<<grid, kAttnTcThreads, smem, st>>>(mq, mk, mv, row_ptr, col_idx, Hq, Hkv, M, causal,
-                                           scale * kLog2e, O, lse);
+                                           group_rows, scale * kLog2e, O, lse);
   return launch_status();
 }
 
 template <bool DENSE>
 int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                 const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C, int block,
-                int causal, float softmax_scale, void* O, float* lse, void* stream) {
+                int causal, float softmax_scale, void* O, float* lse, void* stream,
+                int group_rows = 0) {
   int rc = check_shape(B, Hq, Hkv, M, C, block);
   if (rc != XATTN_OK) return rc;
   if (B == 0 || Hq == 0 || M == 0) return XATTN_OK;
@@ -184,9 +185,9 @@ int attn_common(const void* Q, const void* K, const void* V, const int32_t* row_
   cudaStream_t st = as_stream(stream);
   if (C == 64)
     return launch_attn_tc<64, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
-                                     softmax_scale, o, lse, st);
+                                     group_rows, softmax_scale, o, lse, st);
   return launch_attn_tc<128, DENSE>(q, k, v, row_ptr, col_idx, B, Hq, Hkv, M, causal ? 1 : 0,
-                                    softmax_scale, o, lse, st);
+                                    group_rows, softmax_scale, o, lse, st);
 }
 
 template <bool SELECT = false>
@@ -319,6 +320,54 @@ int xattn_select_ex(const float* scores, const float* param, int rule, int B, in
                        nnz, workspace, workspace_bytes, stream);
 }
 
+size_t xattn_select_group_workspace_size(int B, int Hq, int Hkv, int nb) {
+  if (B < 0 || Hq < 0 || Hkv <= 0 || nb < 0) return 0;
+  const size_t g = (size_t)B * Hkv * nb * sizeof(SelCut);
+  return xattn_select_workspace_size(B, Hq, nb) + ((g + 255) & ~(size_t)255);
+}
+
+int xattn_select_group(const float* scores, const float* param, int rule, int B, int Hq, int Hkv,
+                       int nb, int causal, int32_t* row_ptr, int32_t* col_idx,
+                       size_t col_capacity, int32_t* nnz, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (B < 0 || Hq < 0 || nb < 0 || Hkv <= 0 || Hq % Hkv != 0) return XATTN_EINVAL;
+  if (rule != kSelThreshold && rule != kSelTopK && rule != kSelRatio) return XATTN_EINVAL;
+  if (Hq / Hkv > kSelMaxGroup || nb > kSelMaxNb) return XATTN_EUNSUPPORTED;
+  const long long rows = (long long)B * Hq * nb;
+  const long long grows = (long long)B * Hkv * nb;
+  const long long worst = causal ? grows * (nb + 1) / 2 : grows * nb;
+  if (worst >= (1LL << 31) || rows >= (1LL << 31) - 1) return XATTN_EUNSUPPORTED;
+  if (!row_ptr || !nnz) return XATTN_EINVAL;
+  cudaStream_t st = as_stream(stream);
+  if (rows == 0) {
+    if (cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
+    return XATTN_OK;
+  }
+  if (!scores || !param || !col_idx || !workspace) return XATTN_EINVAL;
+  if (workspace_bytes < xattn_select_group_workspace_size(B, Hq, Hkv, nb)) return XATTN_EINVAL;
+  if (((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
+  SelCut* cuts = static_cast<SelCut*>(workspace);
+  SelCut* gcuts = reinterpret_cast<SelCut*>(static_cast<uint8_t*>(workspace) +
+                                            xattn_select_workspace_size(B, Hq, nb));
+  int P = 1;
+  while (P < nb) P <<= 1;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
+  select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, param, Hq, nb,
+                                                                  causal ? 1 : 0, cuts, rule);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  select_group_count_kernel<<<(unsigned)grows, kSelThreads, 0, st>>>(scores, cuts, Hq, Hkv, nb,
+                                                                     causal ? 1 : 0, gcuts);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
+  select_scan_kernel<<<1, 1024, 0, st>>>(gcuts, (int)grows, row_ptr, nnz, cap);
+  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
+  select_group_fill_kernel<<<(unsigned)grows, kSelThreads, 0, st>>>(
+      scores, cuts, gcuts, Hq, Hkv, nb, causal ? 1 : 0, row_ptr, col_idx);
+  return launch_status();
+}
+
 size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block) {
   const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block);
   if (a == 0 && !(B == 0 || Hq == 0 || M == 0)) return 0;
@@ -429,6 +478,14 @@ int xattn_sparse_attn(const void* Q, const void* K, const void* V, const int32_t
                       int causal, float softmax_scale, void* O, float* lse, void* stream) {
   return attn_common<false>(Q, K, V, row_ptr, col_idx, B, Hq, Hkv, M, C, block, causal,
                             softmax_scale, O, lse, stream);
+}
+
+int xattn_sparse_attn_group(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
+                            const int32_t* col_idx, int B, int Hq, int Hkv, int M, int C,
+                            int block, int causal, float softmax_scale, void* O, float* lse,
+                            void* stream) {
+  return attn_common<false>(Q, K, V, row_ptr, col_idx, B, Hq, Hkv, M, C, block, causal,
+                            softmax_scale, O, lse, stream, 1);
 }
 
 int xattn_dense_attn(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int M,

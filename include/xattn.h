@@ -264,6 +264,38 @@ XATTN_API int xattn_sparse_attn(const void* Q, const void* K, const void* V,
                       float softmax_scale, void* O, float* lse, void* stream);
 
 /*
+ * GQA-shared kept lists - a variant the pages do not define (there every query
+ * head keeps its own minimal set [XA-app]). For GQA models the query heads of
+ * one KV group share the union of their own kept lists, so that one list of
+ * K/V blocks serves the whole group. Each head's own set is contained in the
+ * union, so each head still covers at least its own threshold mass.
+ *
+ * xattn_select_group - every query head's selection exactly as xattn_select_ex
+ * (same rule and param), then per (b, kvh, r) the ascending union over the
+ * heads h with h / (Hq/Hkv) == kvh. CSR over B*Hkv*nb rows: row_ptr has
+ * B*Hkv*nb + 1 entries, row (b*Hkv + kvh)*nb + r. Hq must be a multiple of Hkv
+ * and Hq/Hkv <= 64 (else XATTN_EINVAL / XATTN_EUNSUPPORTED). Capacity and
+ * error behaviour as in xattn_select; worst case B*Hkv*nb*(nb+1)/2 entries
+ * causal, B*Hkv*nb*nb otherwise.
+ */
+XATTN_API size_t xattn_select_group_workspace_size(int B, int Hq, int Hkv, int nb);
+XATTN_API int xattn_select_group(const float* scores, const float* param, int rule, int B,
+                                 int Hq, int Hkv, int nb, int causal, int32_t* row_ptr,
+                                 int32_t* col_idx, size_t col_capacity, int32_t* nnz,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * xattn_sparse_attn_group - xattn_sparse_attn on GQA-shared lists: query head h
+ * of batch b attends over the kept blocks of CSR row (b*Hkv + h/(Hq/Hkv))*nb + r,
+ * as produced by xattn_select_group. Everything else as in xattn_sparse_attn.
+ */
+XATTN_API int xattn_sparse_attn_group(const void* Q, const void* K, const void* V,
+                                      const int32_t* row_ptr, const int32_t* col_idx,
+                                      int B, int Hq, int Hkv, int M, int C, int block,
+                                      int causal, float softmax_scale, void* O, float* lse,
+                                      void* stream);
+
+/*
  * xattn_dense_attn - the same attention with every key block kept (all c <= r
  * when causal, all c otherwise); no CSR. Used as the dense baseline.
  */

@@ -204,3 +204,20 @@ def test_exp2_selftest_rejects_on_host():
     assert xa._lib.xattn_selftest_exp2(FAKE, FAKE, -1, None) == xa.XATTN_EINVAL
     assert xa._lib.xattn_selftest_exp2(None, FAKE, 4, None) == xa.XATTN_EINVAL
     assert xa._lib.xattn_selftest_exp2(None, None, 0, None) == xa.XATTN_OK
+
+
+def test_group_select_rejects_on_host():
+    assert xa.xattn_select_group_workspace_size(1, 4, 2, 8) == \
+        xa.xattn_select_workspace_size(1, 4, 8) + 256
+    base = [FAKE, FAKE, 0, 1, 4, 2, 8, 1, FAKE, FAKE, 1 << 20, FAKE, FAKE, 1 << 30, None]
+    bad = list(base); bad[5] = 3            # Hq not a multiple of Hkv
+    assert xa._lib.xattn_select_group(*bad) == xa.XATTN_EINVAL
+    bad = list(base); bad[2] = 9            # unknown rule
+    assert xa._lib.xattn_select_group(*bad) == xa.XATTN_EINVAL
+    bad = list(base); bad[4], bad[5] = 128, 1   # 128 heads per KV head
+    assert xa._lib.xattn_select_group(*bad) == xa.XATTN_EUNSUPPORTED
+    bad = list(base); bad[13] = 16          # workspace too small
+    assert xa._lib.xattn_select_group(*bad) == xa.XATTN_EINVAL
+    # grouped attention validates shapes like the per-head entry point
+    assert xa._lib.xattn_sparse_attn_group(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 3, 1024, 128, 128,
+                                           1, 0.1, FAKE, None, None) == xa.XATTN_EINVAL

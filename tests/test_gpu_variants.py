@@ -1,13 +1,16 @@
 """GPU parity of the ablation variants the pages compare against: diagonal-pattern
 scoring, and Top-K / fixed-ratio block selection (XAttention summary, "Measured
-effects" table; DuSA rebuttal, Response to Q2)."""
+effects" table; DuSA rebuttal, Response to Q2); the fused score+select entry point;
+and GQA-shared kept lists, a variant the pages do not define."""
+import math
+
 import numpy as np
 import pytest
 import torch
 
 import oracle as orc
 from tests import parity as P
-from tests.gpu_util import device_inputs, small_workload
+from tests.gpu_util import bf16_to_np, csr_to_dict, device_inputs, dict_to_csr, small_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -148,3 +151,80 @@ def test_fused_score_select_equals_two_calls(M, C, Hq, Hkv, S, causal, B):
         assert torch.equal(sc1, sc2)
         assert int(nz2.item()) == n and torch.equal(rp1, rp2)
         assert torch.equal(ci1[:n], ci2[:n])
+
+
+def _select_group(scores_np, param, rule, Hkv, causal):
+    B, Hq, nb, _ = scores_np.shape
+    sc = torch.from_numpy(np.ascontiguousarray(scores_np, dtype=np.float32)).cuda()
+    pr = torch.tensor(param, dtype=torch.float32, device="cuda")
+    row_ptr = torch.empty(B * Hkv * nb + 1, dtype=torch.int32, device="cuda")
+    col = torch.full((xa.max_kept(B, Hkv, nb, causal),), -7, dtype=torch.int32, device="cuda")
+    nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(xa.xattn_select_group_workspace_size(B, Hq, Hkv, nb), dtype=torch.uint8,
+                     device="cuda")
+    xa.xattn_select_group(sc, pr, rule, Hkv, causal, row_ptr, col, nnz, ws)
+    return row_ptr.cpu().numpy(), col.cpu().numpy(), int(nnz.item())
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("nb,B", [(1, 1), (17, 1), (300, 2)])
+def test_group_selection_is_the_union_of_the_heads(causal, nb, B):
+    """GQA-shared lists (a variant): with Top-K (ranking only) bit-exact against
+    the oracle's union; with the threshold rule, exactly the union of the lists
+    the per-head entry point returns on the same scores."""
+    Hq, Hkv = 4, 2
+    rng = np.random.default_rng(nb * 7 + B + causal)
+    s = rng.gamma(0.3, size=(B, Hq, nb, nb))
+    if causal:
+        s = np.tril(s)
+    s = (s / s.sum(-1, keepdims=True)).astype(np.float32)
+    s64 = s.astype(np.float64)
+    k_param = [3.0, 1.0, 5.0, 2.0]
+    rp, col, nnz = _select_group(s, k_param, xa.XATTN_SELECT_TOPK, Hkv, causal)
+    assert rp[0] == 0 and rp[-1] == nnz
+    kept = {(b, h): {r: orc.select_row_topk(s64[b, h, r], r, int(k_param[h]), causal)
+                     for r in range(nb)} for b in range(B) for h in range(Hq)}
+    union = orc.layer_select_group(kept, Hq, Hkv)
+    for b in range(B):
+        for kvh in range(Hkv):
+            got = csr_to_dict(rp, col, b * Hkv + kvh, nb)
+            for r in range(nb):
+                assert got[r].tolist() == union[(b, kvh)][r].tolist(), (b, kvh, r)
+    tau = [0.9, 0.6, 0.95, 0.8]
+    rp, col, nnz = _select_group(s, tau, xa.XATTN_SELECT_THRESHOLD, Hkv, causal)
+    hrp, hcol, _ = _select_ex(s, tau, xa.XATTN_SELECT_THRESHOLD, causal)
+    per_head = {(b, h): csr_to_dict(hrp, hcol, b * Hq + h, nb) for b in range(B) for h in range(Hq)}
+    union = orc.layer_select_group(per_head, Hq, Hkv)
+    for b in range(B):
+        for kvh in range(Hkv):
+            got = csr_to_dict(rp, col, b * Hkv + kvh, nb)
+            for r in range(nb):
+                assert got[r].tolist() == union[(b, kvh)][r].tolist(), (b, kvh, r)
+    assert nnz == sum(len(v[r]) for v in union.values() for r in range(nb))
+
+
+@pytest.mark.parametrize("M,C,Hq,Hkv,causal", [
+    (1536, 128, 4, 2, True),
+    (1152, 64, 4, 1, False),
+])
+def test_group_attention_matches_oracle(M, C, Hq, Hkv, causal):
+    """Attention over GQA-shared lists: every head of a group attends over the
+    group's union list."""
+    w = small_workload(M, C, Hq, Hkv, 8, causal)
+    (Qb, Kb, Vb), (Q, K, V) = device_inputs(w)
+    nb = M // 128
+    sig = orc.default_score_scale(8, C)
+    sc = orc.layer_block_scores(Qb, Kb, Hkv, 8, 128, sig, causal)
+    kept = orc.layer_select(sc, np.full(Hq, 0.7), causal)
+    union = orc.layer_select_group(kept, Hq, Hkv)
+    row_ptr, col = dict_to_csr(union, 1, Hkv, nb)
+    O = torch.empty_like(Q)
+    lse = torch.empty((1, Hq, M), device="cuda")
+    xa.xattn_sparse_attn_group(Q, K, V, row_ptr, col, causal, 1 / math.sqrt(C), O, lse)
+    grp = Hq // Hkv
+    by_head = {(0, h): union[(0, h // grp)] for h in range(Hq)}
+    ref = orc.layer_sparse_attention(Qb, Kb, Vb, Hkv, by_head, 128, causal, 1 / math.sqrt(C))
+    got, glse = bf16_to_np(O), lse.cpu().numpy()
+    for h in range(Hq):
+        P.assert_outputs_close(got[0, h], ref[(0, h)][0], f"O head {h}")
+        np.testing.assert_allclose(glse[0, h], ref[(0, h)][1], rtol=1e-4, atol=1e-4)
