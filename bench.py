@@ -379,6 +379,13 @@ def main():
         "dense_equivalent_tflops": dense_eq_flops / (ms_step * 1e-3) / 1e12,
         # fused: the score stage also holds the row ranking, scan and fill
         "score_tflops": score_flops / (st_score * 1e-3) / 1e12,
+        "score_frac_of_bf16_peak": score_flops / (st_score * 1e-3) / 1e12 / pk["bf16_sustained"],
+        # selection (count + scan + fill): reads the candidate scores, writes
+        # row_ptr and the kept lists; HBM-bound by design
+        "select_gbs": (4.0 * (cand + nnz + w.B * w.Hq * w.nb) / (st_select * 1e-3) / 1e9
+                       if st_select > 0 else None),
+        # secondary ceiling of the attention: b^2 exponentials per kept block
+        "attn_exp2_per_s": w.block ** 2 * nnz / (st_attn * 1e-3),
     }
 
     # dense baseline (the build's own dense attention), same inputs
