@@ -8,28 +8,34 @@
 //   warp 0, one lane  TMA producer: Q once, then the K and V tiles of the kept
 //                     blocks (in list order) into two rings of kStages stages with
 //                     their own full/empty barriers; K runs one block ahead of V.
-//   warp 1, one lane  S issuer and TMEM owner: S = Q K^T into one of three TMEM
+//   warp 1, one lane  S issuer and TMEM owner: S = Q K^T into one of two TMEM
 //                     buffers (128 lanes x 128 fp32 columns each); S of block j
-//                     goes to buffer j%3 as soon as the PV MMAs of block j-3,
-//                     which read P from that buffer, have completed, so the S of
-//                     the next two blocks is computed while the softmax works on
-//                     this one and the PV of a block is off the softmax's path.
-//   warp 2, one lane  PV issuer (on its own sub-partition, apart from the S
-//                     issuer): O += P V into one TMEM accumulator once both halves
-//                     of the block's P are written.
+//                     goes to buffer j%2 as soon as the PV MMAs of block j-2,
+//                     which read P from that buffer, have completed, so the next
+//                     block's S is computed while the softmax works on this one.
+//   warps 2, 3,       PV issuers, one per key half g (keys 64g..64g+63):
+//   one lane each     O_g += P_g V_g into the half's own TMEM accumulator, as soon
+//                     as that half's P is written. Issuing is split over three
+//                     threads on different sub-partitions because one thread
+//                     cannot issue the 16 MMAs of a block and poll their barriers
+//                     as fast as the tensor core retires them, and so that one
+//                     half's PV never queues behind the other's; each issuer's
+//                     commits track exactly its own MMAs.
 //   warps 4-11        softmax, two threads per query row (TMEM lane = row): warps
 //                     4-7 own keys 0-63 of every block, warps 8-11 keys 64-127.
-//                     Both threads of a row read the whole row of S and take its
-//                     max, so they hold the same running max without talking to
-//                     each other, and each exponentiates its own half. Per block:
-//                     causal mask on the diagonal block, fp32 base-2 softmax with
-//                     the scale folded into one FMA, lazy rescaling (O and l are
-//                     rescaled only when the running max grows by more than 2^8;
-//                     each thread rescales its half of O's columns), P_g as bf16
-//                     over the first 32 columns of its half of the S buffer, where
-//                     the PV MMA reads it as its A operand. Only a rescale waits
-//                     for the previous block's PV. At the end the two halves' sums
-//                     are added and each thread writes half of the row of O / l.
+//                     The two halves are independent online softmaxes over
+//                     disjoint key sets (own running max m_g, sum l_g, accumulator
+//                     O_g), so they never wait for each other inside the loop; at
+//                     the end they are merged exactly:
+//                       m = max(m_0, m_1), l = sum_g l_g 2^(m_g - m),
+//                       O = sum_g O_g 2^(m_g - m) / l.
+//                     Per block: read the half row of S, causal mask on the
+//                     diagonal block, fp32 base-2 softmax with the scale folded into
+//                     one FMA, lazy rescaling (O_g and l_g are rescaled only when
+//                     m_g grows by more than 2^8), P_g as bf16 over the first 32
+//                     columns of its own half of the S buffer, where the PV MMA
+//                     reads it as its A operand. Only a rescale waits for the
+//                     previous block's PV.
 // Every role walks the row's list with the next entry's load already in flight
 // (ListIter), so no role waits on a global load inside its loop.
 // Every wait is bounded (sm100::mbar_wait); on a timeout the CTA raises
@@ -43,7 +49,7 @@ namespace xattn {
 
 constexpr int kAttnTcThreads = 384;
 #ifndef XATTN_EXP2_EMU_PER4
-#define XATTN_EXP2_EMU_PER4 1
+#define XATTN_EXP2_EMU_PER4 2
 #endif
 constexpr int kEmuPer4 = XATTN_EXP2_EMU_PER4;   // softmax pairs (of 4) on the FMA pipe
 
@@ -59,10 +65,9 @@ struct AttnTc {
   static constexpr int kOffBar = kOffV + kStages * kTile;
   static constexpr int kOffX = kOffBar + 256;             // end-of-row (m, l) exchange
   static constexpr int kSmem = kOffX + 2 * 128 * 8 + 1024;  // + alignment slack
-  static constexpr int kTmemCols = 512;                   // S_0, S_1, S_2, O
-  static constexpr int kNumS = 3;                         // S buffers
+  static constexpr int kTmemCols = 512;                   // S_0, S_1, O_0, O_1
   static constexpr int kColS = 0;                         // + b * 128: 128 fp32 columns each
-  static constexpr int kColO = 384;                       // C fp32 columns
+  static constexpr int kColO = 256;                       // + g * 128: C fp32 columns each
   // P_g of the block in S buffer b: 64 bf16 keys packed into the first 32
   // columns of that buffer's half g (kColS + b * 128 + g * 64)
 };
@@ -114,15 +119,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* k_full = bars;            // [ST] K tile of a block landed
   uint64_t* k_empty = bars + ST;      // [ST] its S MMA completed
   uint64_t* v_full = bars + 2 * ST;   // [ST] V tile of a block landed
-  uint64_t* v_empty = bars + 3 * ST;  // [ST] its PV MMAs completed
+  uint64_t* v_empty = bars + 3 * ST;  // [ST] both of its PV MMAs completed (2 issuers)
   uint64_t* q_full = bars + 4 * ST;
-  uint64_t* s_full = q_full + 1;      // [3 buffers] S of the block computed
-  uint64_t* s_free = q_full + 4;      // [3 buffers] the PV MMAs reading P from it completed
-  uint64_t* p_full = q_full + 7;      // [3 buffers] both halves of P written (8 warps)
-  uint64_t* o_done = q_full + 10;     // PV of the block completed
-  uint64_t* drain = q_full + 11;      // [2] S issuer, PV issuer
-  uint64_t* x_full = q_full + 13;     // end-of-row sums l_g published (8 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 14);
+  uint64_t* s_full = q_full + 1;      // [2 buffers] S of the block computed
+  uint64_t* s_free = q_full + 3;      // [2 buffers] both PV MMAs reading P from it completed (2)
+  uint64_t* p_full = q_full + 5;      // [2 halves][2 buffers] P_g written (4 warps each)
+  uint64_t* o_done = q_full + 9;      // [2 halves] PV_g of the block completed
+  uint64_t* drain = q_full + 11;      // [3] S issuer, PV issuers of halves 0 and 1
+  uint64_t* x_full = q_full + 14;     // end-of-row (m_g, l_g) published (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float2* xchg = reinterpret_cast<float2*>(smem + L::kOffX);   // [2 half][128]
 
@@ -140,14 +145,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (tid == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 2);
     }
     mbar_init(q_full, 1);
-    for (int i = 0; i < L::kNumS; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 1); mbar_init(&p_full[i], 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 2);
+      mbar_init(&p_full[2 * i], 4); mbar_init(&p_full[2 * i + 1], 4);
+      mbar_init(&o_done[i], 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(&drain[0], 1); mbar_init(&drain[1], 1);
+    mbar_init(&drain[0], 1); mbar_init(&drain[1], 1); mbar_init(&drain[2], 1);
     mbar_init(x_full, 8);
     *abort_flag = 0;
     fence_mbar_init();
@@ -213,7 +219,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int jj = (nv > ST ? nv - ST : 0); jj < nv; ++jj)
         mbar_wait(&v_full[jj % ST], (jj / ST) & 1, &no_abort);
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp >= 1 && warp <= 3) {
     // ------------------------------------------------- S and PV issuers
     if (lane == 0) {
       // descriptors built once; per MMA only the start address (16-byte units,
@@ -232,21 +238,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         auto issue_S = [&](int j) {
           const int st = j % ST;
           const uint64_t dKs = dK + (uint64_t)((st * L::kTile) >> 4);
-          const uint32_t tSb = tmem + L::kColS + (j % L::kNumS) * 128;
+          const uint32_t tSb = tmem + L::kColS + (j & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * L::kRegion + (kk & 3) * 32) >> 4;
             mma_f16_ss(tSb, dQ + off, dKs + off, idS, kk > 0);
           }
-          mma_commit(&s_full[j % L::kNumS]);
+          mma_commit(&s_full[j & 1]);
           mma_commit(&k_empty[st]);
         };
         ok = have_cur && mbar_wait(q_full, 0, abort_flag);
         for (int j = 0; ok && have_cur; ++j) {
-          // buffer j%3 is free once the PV MMAs of block j-3 have read its P
+          // buffer j%2 is free once the PV MMAs of block j-2 have read its P
           ok = mbar_wait(&k_full[j % ST], (j / ST) & 1, abort_flag) &&
-               (j < L::kNumS ||
-                mbar_wait(&s_free[j % L::kNumS], ((j / L::kNumS) - 1) & 1, abort_flag));
+               (j < 2 || mbar_wait(&s_free[j & 1], ((j >> 1) - 1) & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
           issue_S(j);
@@ -254,23 +259,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           have_nxt = have_cur && li.next() >= 0;
         }
       } else {
+        const int g = warp - 2;              // key half of this PV issuer
         for (int j = 0; ok && have_cur; ++j) {
           const int st = j % ST;
-          const int b = j % L::kNumS;
+          const int b = j & 1;
           if (!(ok = mbar_wait(&v_full[st], (j / ST) & 1, abort_flag) &&
-                     mbar_wait(&p_full[b], (j / L::kNumS) & 1, abort_flag)))
+                     mbar_wait(&p_full[2 * g + b], (j >> 1) & 1, abort_flag)))
             break;
           tc_fence_after();
-          const uint64_t dVs = dV + (uint64_t)((st * L::kTile) >> 4);
+          const uint64_t dVg = dV + (uint64_t)((st * L::kTile + g * 4 * 2048) >> 4);
+          const uint32_t tP = tmem + L::kColS + b * 128 + g * 64;
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const uint32_t tP = tmem + L::kColS + b * 128 + g * 64;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)   // keys 64g + 16kk .. +15 (8 TMEM columns)
-              mma_f16_ts(tmem + L::kColO, tP + kk * 8, dVs + ((g * 4 + kk) * 2048 >> 4), idPV,
-                         (j > 0 || g > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(o_done);
+          for (int kk = 0; kk < 4; ++kk)     // keys 64g + 16kk .. +15 (8 TMEM columns)
+            mma_f16_ts(tmem + L::kColO + g * 128, tP + kk * 8, dVg + (kk * 2048 >> 4), idPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&o_done[g]);
           mma_commit(&v_empty[st]);
           mma_commit(&s_free[b]);
           have_cur = have_nxt;
@@ -287,50 +290,41 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int g = (warp >= 8) ? 1 : 0;                 // keys [64g, 64g + 64) of each block
     const int q_row = (warp & 3) * 32 + lane;          // row within the query block
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tSg = tmem + lane_off + L::kColS + g * 64;        // + b * 128
-    const uint32_t tSo = tmem + lane_off + L::kColS + (1 - g) * 64;  // the other half
-    const uint32_t tOg = tmem + lane_off + L::kColO + g * (C / 2);   // this half of O
-    const int k0 = g * 64, k1 = (1 - g) * 64;
+    const uint32_t tSg = tmem + lane_off + L::kColS + g * 64;   // + b * 128
+    const uint32_t tOg = tmem + lane_off + L::kColO + g * 128;
+    const int k0 = g * 64;
     float m = kNegInf, l = 0.f;
     int j = 0;
     bool ok = true;
     ListIter li;
     li.init(col_idx, beg, end, nb, r, causal != 0, DENSE);
     for (int c = li.next(); c >= 0; c = li.next()) {
-      const int b = j % L::kNumS;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j / L::kNumS) & 1, abort_flag));
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float s[64], so[64];
+      float s[64];
       tmem_ld32(tSg + b * 128, s);
       tmem_ld32(tSg + b * 128 + 32, s + 32);
-      tmem_ld32(tSo + b * 128, so);
-      tmem_ld32(tSo + b * 128 + 32, so + 32);
       tmem_wait_ld();
 
-      // max of the whole row of raw logits (the scale is positive), the same
-      // value in both threads of the row; masked keys of the diagonal block are
-      // set to -inf first, on the diagonal block only
+      // half-row max of the raw logits (the scale is positive); masked keys of
+      // the diagonal block are set to -inf first, on the diagonal block only
       if (causal && c == r) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          s[i] = (k0 + i > q_row) ? kNegInf : s[i];
-          so[i] = (k1 + i > q_row) ? kNegInf : so[i];
-        }
+        for (int i = 0; i < 64; ++i) s[i] = (k0 + i > q_row) ? kNegInf : s[i];
       }
       // eight independent partial maxima / sums keep the reductions off one
       // long dependency chain; three-input max and packed fp32x2 FMA / add halve
       // the instruction count of the two reductions and of the exponent arguments
       float pm[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) pm[k] = fmax3(s[k], so[k], so[k + 8]);
+      for (int k = 0; k < 8; ++k) pm[k] = s[k];
 #pragma unroll
       for (int i = 8; i < 64; i += 2) pm[(i >> 1) & 7] = fmax3(pm[(i >> 1) & 7], s[i], s[i + 1]);
-#pragma unroll
-      for (int i = 16; i < 64; i += 2) pm[(i >> 1) & 7] = fmax3(pm[(i >> 1) & 7], so[i], so[i + 1]);
       const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]),
                              fmaxf(pm[6], pm[7]));
-      // a row may see no key yet (the first rows of a diagonal-only list)
+      // a row may see no key of this half (the upper half of the diagonal block)
       const float m_new = fmaxf(m, mx * scale_log2);
       float corr = 1.f;
       bool resc = false;
@@ -364,14 +358,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float rs = pq.x + pq.y;
       l = l * corr + rs;
 
-      // a rescale needs O stable: the previous block's PV complete; each thread
-      // of the row rescales its half of O's columns
+      // a rescale needs O_g stable: PV_g of the previous block complete
       if (__any_sync(0xffffffffu, resc)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[g], (j - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < C / 64; ++q) {
+        for (int q = 0; q < C / 32; ++q) {
           float o[32];
           tmem_ld32(tOg + q * 32, o);
           tmem_wait_ld();
@@ -392,13 +385,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[b]);
+      if (lane == 0) mbar_arrive(&p_full[2 * g + b]);
       ++j;
     }
 
-    // the last PV, then the row sum l = l_0 + l_1 (both halves use the same m)
+    // last PV of this half, then merge the halves: publish (m_g, l_g)
     if (ok && j > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_done[g], (j - 1) & 1, abort_flag));
     }
     if (ok) {
       xchg[g * 128 + q_row] = make_float2(m, l);
@@ -407,33 +400,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ok = __all_sync(0xffffffffu, mbar_wait(x_full, 0, abort_flag));
     }
     if (ok) {
-      tc_fence_after();
-      const float lt = xchg[q_row].y + xchg[128 + q_row].y;
+      tc_fence_after();   // the other half's last PV completed before it arrived
+      const float2 s0 = xchg[q_row], s1 = xchg[128 + q_row];
+      const bool has0 = s0.y > 0.f, has1 = s1.y > 0.f;
+      const float mm = fmaxf(has0 ? s0.x : kNegInf, has1 ? s1.x : kNegInf);
+      const float f0 = has0 ? ex2(s0.x - mm) : 0.f;
+      const float f1 = has1 ? ex2(s1.x - mm) : 0.f;
+      const float lt = s0.y * f0 + s1.y * f1;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       // this half writes output columns [g*C/2, (g+1)*C/2)
       bf16* orow = O + ((size_t)bh * M + (size_t)r * 128 + q_row) * C + g * (C / 2);
+      const uint32_t tO0 = tmem + lane_off + L::kColO + g * (C / 2);
 #pragma unroll
       for (int q = 0; q < C / 64; ++q) {
-        float a[32];
-        if (j > 0) {
-          tmem_ld32(tOg + q * 32, a);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = 0.f;
-        }
+        float a0[32], a1[32];
+        tmem_ld32(tO0 + q * 32, a0);
+        tmem_ld32(tO0 + 128 + q * 32, a1);
+        tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
+          float vv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            vv[e] = ((has0 ? a0[i + e] * f0 : 0.f) + (has1 ? a1[i + e] * f1 : 0.f)) * inv;
           uint4 v;
-          v.x = pack_bf16x2(a[i] * inv, a[i + 1] * inv);
-          v.y = pack_bf16x2(a[i + 2] * inv, a[i + 3] * inv);
-          v.z = pack_bf16x2(a[i + 4] * inv, a[i + 5] * inv);
-          v.w = pack_bf16x2(a[i + 6] * inv, a[i + 7] * inv);
+          v.x = pack_bf16x2(vv[0], vv[1]);
+          v.y = pack_bf16x2(vv[2], vv[3]);
+          v.z = pack_bf16x2(vv[4], vv[5]);
+          v.w = pack_bf16x2(vv[6], vv[7]);
           *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
         }
       }
       if (lse != nullptr && g == 0)
-        lse[(size_t)bh * M + (size_t)r * 128 + q_row] = lt > 0.f ? (m + lg2(lt)) * kLn2 : kNegInf;
+        lse[(size_t)bh * M + (size_t)r * 128 + q_row] = lt > 0.f ? (mm + lg2(lt)) * kLn2 : kNegInf;
     }
     tc_fence_before();
   }
