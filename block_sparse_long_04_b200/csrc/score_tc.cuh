@@ -17,13 +17,13 @@
 //
 // Warp roles (256 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA
 // issuer (warp 1 also owns the TMEM allocation), warps 4-7 = epilogue, one
-// reshaped row per thread (TMEM lane = row).
+// reshaped row per thread (TMEM lane = row); all eight warps share the finalize.
 //
 // Epilogue (row softmax + block summation, XAttention summary, Approach): for
 // every key block of g = 128/S columns the thread forms the block's base-2
 // log-sum-exp ell[i', c] from its TMEM row, updates the row's running LSE, and
-// writes ell to the workspace. After the sweep the same threads re-read their
-// CTA's ell values (L2-resident) and write
+// writes ell to the workspace. After the sweep all threads of the CTA re-read its
+// ell values (L2-resident) and write
 //   scores[r, c] = (1/g) sum_{i' in r} 2^(ell[i', c] - LSE[i']).
 // The (M/S)^2 logits are never stored. Waits are bounded as in attn_tc.cuh.
 //
@@ -217,61 +217,64 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
 
-    // ---- finalize among the 128 epilogue threads (named barrier 1) ----
+    // ---- row LSE, then the finalize by all warps ----
     if (ok) {
       const float L_row = (l_run > 0.f) ? m_run + lg2(l_run) : kNegInf;
       lse_s[rl] = L_row;
       if (ip < rp) lse_ws[(size_t)bh * rp + ip] = L_row;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok && !*abort_flag) {
-      const int et = tid - 128;
-      const float inv_g = 1.f / (float)G;
-      for (int k = 0; k < 128 / G; ++k) {
-        const int r = i0 / G + k;
-        if (r >= nb) break;
-        const int ncand = causal ? r + 1 : nb;
-        float* srow = scores + ((size_t)bh * nb + r) * nb;
-        const float* pr0 = part + ((size_t)bh * rp + (size_t)r * G) * nb;
-        for (int c = et; c < nb; c += 128) {
-          float acc = 0.f;
-          if (c < ncand) {
+    tc_fence_before();
+  }
+
+  // The producer and MMA warps are idle by now, so all 256 threads turn the
+  // partials of the CTA's rows into block scores (a wait that failed has set
+  // the abort flag, which every thread reads after the barrier).
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+  const bool done_ok = !*abort_flag;
+  if (done_ok) {
+    const float inv_g = 1.f / (float)G;
+    for (int k = 0; k < 128 / G; ++k) {
+      const int r = i0 / G + k;
+      if (r >= nb) break;
+      const int ncand = causal ? r + 1 : nb;
+      float* srow = scores + ((size_t)bh * nb + r) * nb;
+      const float* pr0 = part + ((size_t)bh * rp + (size_t)r * G) * nb;
+      for (int c = tid; c < nb; c += kScoreTcThreads) {
+        float acc = 0.f;
+        if (c < ncand) {
 #pragma unroll 4
-            for (int i = 0; i < G; ++i) acc += ex2(pr0[(size_t)i * nb + c] - lse_s[r * G + i - i0]);
-            acc *= inv_g;
-          }
-          srow[c] = acc;
+          for (int i = 0; i < G; ++i) acc += ex2(pr0[(size_t)i * nb + c] - lse_s[r * G + i - i0]);
+          acc *= inv_g;
         }
+        srow[c] = acc;
       }
     }
-    if (SELECT) {
-      // fused selection of the rows just written; one uniform decision first
-      volatile int* go = reinterpret_cast<volatile int*>(lse_s + 128);
-      if (tid == 128) *go = (ok && !*abort_flag) ? 1 : 0;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (*go) {
-        const int et = tid - 128;
-        float* key = reinterpret_cast<float*>(smem);                    // the idle stage ring
-        int* idx = reinterpret_cast<int*>(smem + kSelMaxNb * 4);
+  }
+  if (SELECT) {
+    // fused selection of the rows just written, by the 128 epilogue threads
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (warp >= 4) {
+      const int et = tid - 128;
+      if (done_ok) {
+        uint64_t* keys = reinterpret_cast<uint64_t*>(smem);             // the idle stage ring
         double* red = reinterpret_cast<double*>(smem + kSelMaxNb * 8);
         int* first_hit = reinterpret_cast<int*>(red + 4);
-        auto sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+        auto sync = [] { asm volatile("bar.sync 2, 128;" ::: "memory"); };
         for (int k = 0; k < 128 / G; ++k) {
           const int r = i0 / G + k;
           if (r >= nb) break;
           const int n = causal ? r + 1 : nb;
           const SelCut cut = select_row_cut<128>(scores + ((size_t)bh * nb + r) * nb, n, r,
-                                                 sel_param[h], sel_rule, key, idx, red,
+                                                 sel_param[h], sel_rule, keys, red,
                                                  first_hit, et, sync);
           if (et == 0) cuts[(size_t)bh * nb + r] = cut;
         }
       } else {
         // no scores: empty cuts, so the scan and fill passes write nothing for these rows
-        const int r = i0 / G + (tid - 128);
-        if (tid - 128 < 128 / G && r < nb) cuts[(size_t)bh * nb + r] = SelCut{0.f, 0, 0};
+        const int r = i0 / G + et;
+        if (et < 128 / G && r < nb) cuts[(size_t)bh * nb + r] = SelCut{0.f, 0, 0};
       }
     }
-    tc_fence_before();
   }
 
   __syncthreads();

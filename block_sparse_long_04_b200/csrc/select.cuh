@@ -69,6 +69,17 @@ __device__ __forceinline__ int block_exclusive_scan_i32(int v, int* red, int& to
   return before;
 }
 
+// 32-bit rank of a score for an ascending sort that puts higher scores first:
+// the float bits mapped to an order-preserving unsigned, then inverted.
+__device__ __forceinline__ uint32_t desc_rank(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return ~((u & 0x80000000u) ? ~u : (u | 0x80000000u));
+}
+__device__ __forceinline__ float rank_score(uint32_t rk) {
+  const uint32_t o = ~rk;
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
 // Exclusive scan of one fp64 value per thread over a group of NT threads (whole
 // warps) that share `sync` as their barrier; red holds NT/32 doubles.
 template <int NT, typename Sync>
@@ -89,37 +100,34 @@ __device__ __forceinline__ double group_exclusive_scan_f64(double v, double* red
 }
 
 // The cut of one row of block scores (candidates 0..n-1, diagonal r), computed
-// by a group of NT threads: bitonic sort of (score, index) keys in shared memory
-// (descending score, ascending index), then the cut position of the rule: the
-// first prefix whose fp64 cumulative sum reaches t (threshold), floor(t) (Top-K)
-// or ceil(t * n) (ratio), clamped to [1, n]. key/idx hold P floats / ints with
-// P = next power of two >= n. The result is valid in thread 0 of the group.
+// by a group of NT threads: bitonic sort of 64-bit keys (descending-score rank,
+// then index) in shared memory, i.e. descending score, ascending index; then the
+// cut position of the rule: the first prefix whose fp64 cumulative sum reaches t
+// (threshold), floor(t) (Top-K) or ceil(t * n) (ratio), clamped to [1, n]. keys
+// holds P entries, P = next power of two >= n. The result is valid in thread 0
+// of the group.
 template <int NT, typename Sync>
 __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, float t, int rule,
-                                 float* key, int* idx, double* red, int* first_hit, int tid,
-                                 Sync sync) {
+                                 uint64_t* keys, double* red, int* first_hit, int tid, Sync sync) {
   int P = 1;
   while (P < n) P <<= 1;
-  for (int i = tid; i < P; i += NT) {
-    key[i] = i < n ? srow[i] : kNegInf;
-    idx[i] = i < n ? i : 0x7fffffff;
-  }
+  for (int i = tid; i < P; i += NT)
+    keys[i] = i < n ? ((uint64_t)desc_rank(srow[i]) << 32) | (uint32_t)i
+                    : ((uint64_t)desc_rank(kNegInf) << 32) | 0x7fffffffu;
   if (tid == 0) *first_hit = n - 1;
   sync();
 
-  // bitonic network: ascending "rank" order = descending score, ascending index
+  // bitonic network over one 64-bit word per entry (one load and one store per
+  // side instead of separate score and index arrays)
   for (int k = 2; k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       for (int i = tid; i < P; i += NT) {
         const int p = i ^ j;
         if (p > i) {
-          const float si = key[i], sp = key[p];
-          const int ii = idx[i], ip = idx[p];
-          const bool i_first = ranks_before(si, ii, sp, ip);
-          const bool up = (i & k) == 0;
-          if (up != i_first) {
-            key[i] = sp; key[p] = si;
-            idx[i] = ip; idx[p] = ii;
+          const uint64_t a = keys[i], b = keys[p];
+          if ((a > b) == ((i & k) == 0)) {
+            keys[i] = b;
+            keys[p] = a;
           }
         }
       }
@@ -140,11 +148,11 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   const int per = (n + NT - 1) / NT;
   const int lo = tid * per, hi = min(n, lo + per);
   double seg = 0.0;
-  for (int i = lo; i < hi; ++i) seg += (double)key[i];
+  for (int i = lo; i < hi; ++i) seg += (double)rank_score((uint32_t)(keys[i] >> 32));
   double run = group_exclusive_scan_f64<NT>(seg, red, tid, sync);
   if (rule == kSelThreshold && t < 1.0f) {
     for (int i = lo; i < hi; ++i) {
-      run += (double)key[i];
+      run += (double)rank_score((uint32_t)(keys[i] >> 32));
       if (run >= (double)t) { atomicMin(first_hit, i); break; }
     }
   }
@@ -152,8 +160,8 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   SelCut cut;
   if (tid == 0) {
     const int k = *first_hit;
-    cut.score = key[k];
-    cut.index = idx[k];
+    cut.score = rank_score((uint32_t)(keys[k] >> 32));
+    cut.index = (int)(uint32_t)keys[k];
     const bool diag_kept = r == cut.index || ranks_before(srow[r], r, cut.score, cut.index);
     cut.count = k + 1 + (diag_kept ? 0 : 1);
   }
@@ -177,10 +185,9 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
   const int n = causal ? r + 1 : nb;
   int P = 1;
   while (P < n) P <<= 1;
-  float* key = reinterpret_cast<float*>(smem);
-  int* idx = reinterpret_cast<int*>(smem + (size_t)P * 4);
-  const SelCut cut = select_row_cut<kSelThreads>(scores + (size_t)row * nb, n, r, tau[h], rule, key,
-                                                 idx, red, &first_hit, (int)threadIdx.x,
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
+  const SelCut cut = select_row_cut<kSelThreads>(scores + (size_t)row * nb, n, r, tau[h], rule,
+                                                 keys, red, &first_hit, (int)threadIdx.x,
                                                  [] { __syncthreads(); });
   if (threadIdx.x == 0) cuts[row] = cut;
 }
