@@ -99,6 +99,67 @@ __device__ __forceinline__ double group_exclusive_scan_f64(double v, double* red
   return before;
 }
 
+// Ascending bitonic sort of P = 256 * E 64-bit keys by 256 threads, thread t
+// holding entries tE .. tE+E-1 in registers: compare-exchange partners at
+// distance j < E are in the same thread, at E <= j < 32E in the same warp (a
+// shuffle), and only the stages with j >= 32E go through shared memory. Each
+// entry keeps the minimum of its pair when it is the pair's lower entry in an
+// ascending run (or the upper one in a descending run), else the maximum.
+template <int E>
+__device__ __forceinline__ void bitonic_sort_256(uint64_t* keys, int tid) {
+  constexpr int P = 256 * E;
+  uint64_t v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = keys[tid * E + e];
+#pragma unroll 1
+  for (int k = 2; k <= P; k <<= 1) {
+    // partners in other threads: shared memory or a shuffle
+#pragma unroll 1
+    for (int j = k >> 1; j >= E; j >>= 1) {
+      if (j >= 32 * E) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) keys[tid * E + e] = v[e];
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const uint64_t o = keys[i ^ j];
+          const bool take_min = ((i & j) == 0) == ((i & k) == 0);
+          v[e] = take_min ? (o < v[e] ? o : v[e]) : (o > v[e] ? o : v[e]);
+        }
+        __syncthreads();
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], j / E);
+          const bool take_min = ((i & j) == 0) == ((i & k) == 0);
+          v[e] = take_min ? (o < v[e] ? o : v[e]) : (o > v[e] ? o : v[e]);
+        }
+      }
+    }
+    // partners in the same thread (distance jj < E, known at compile time)
+#pragma unroll
+    for (int jj = E / 2; jj > 0; jj >>= 1) {
+      if (jj < k) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          if ((e & jj) == 0) {
+            const int i = tid * E + e;
+            const uint64_t a = v[e], b = v[e ^ jj];
+            if ((a > b) == ((i & k) == 0)) {
+              v[e] = b;
+              v[e ^ jj] = a;
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) keys[tid * E + e] = v[e];
+}
+
 // The cut of one row of block scores (candidates 0..n-1, diagonal r), computed
 // by a group of NT threads: bitonic sort of 64-bit keys (descending-score rank,
 // then index) in shared memory, i.e. descending score, ascending index; then the
@@ -118,8 +179,21 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   sync();
 
   // bitonic network over one 64-bit word per entry (one load and one store per
-  // side instead of separate score and index arrays)
-  for (int k = 2; k <= P; k <<= 1) {
+  // side instead of separate score and index arrays); 256-thread groups sort
+  // rows of 256 to 2048 entries mostly in registers
+  bool sorted = false;
+  if (NT == 256 && P >= 256) {
+    sorted = true;
+    switch (P / 256) {
+      case 1: bitonic_sort_256<1>(keys, tid); break;
+      case 2: bitonic_sort_256<2>(keys, tid); break;
+      case 4: bitonic_sort_256<4>(keys, tid); break;
+      case 8: bitonic_sort_256<8>(keys, tid); break;
+      default: sorted = false;   // longer rows: the shared-memory network below
+    }
+    sync();
+  }
+  for (int k = 2; !sorted && k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       for (int i = tid; i < P; i += NT) {
         const int p = i ^ j;
