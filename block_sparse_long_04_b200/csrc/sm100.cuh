@@ -1,5 +1,5 @@
-// sm_100a primitives: mbarriers with bounded waits, TMA tile loads (no cluster
-// multicast), tcgen05 (TMEM allocation, MMA, commit, TMEM loads/stores) and the
+// sm_100a primitives: mbarriers with bounded waits, TMA tile loads (each CTA
+// loads its own tiles), tcgen05 (TMEM allocation, MMA, commit, TMEM loads/stores) and the
 // shared-memory / instruction descriptors the tensor core reads.
 #pragma once
 #include <cuda.h>
