@@ -103,19 +103,33 @@ def peaks():
 
 # ------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs.
+
+    nvidia-smi takes a few hundred ms to start, so the sampler is started before
+    the warm-up and every sample carries its arrival time; summary() keeps the
+    samples that arrived between mark_start() and mark_end() (plus one sampling
+    period of slack at the end)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    PERIOD_MS = 50
+
     def __init__(self, index):
         self.index, self.rows, self.proc = index, [], None
+        self.t_start, self.t_end = None, None
+
+    def mark_start(self):
+        self.t_start = time.monotonic()
+
+    def mark_end(self):
+        self.t_end = time.monotonic()
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-i", str(self.index), "-lms", "100"], stdout=subprocess.PIPE,
+                 "-i", str(self.index), "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -125,7 +139,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.rows.append([x.strip() for x in line.split(",")])
+            self.rows.append((time.monotonic(), [x.strip() for x in line.split(",")]))
 
     def __exit__(self, *exc):
         if self.proc:
@@ -136,15 +150,21 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.rows:
+        rows = self.rows
+        if self.t_start is not None and self.t_end is not None:
+            slack = self.PERIOD_MS / 1000.0
+            rows = [r for t, r in rows if self.t_start <= t <= self.t_end + slack]
+        else:
+            rows = [r for _, r in rows]
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.rows)}
+                "samples": len(rows)}
 
 
 # --------------------------------------------------------- CPU oracle sample
@@ -326,22 +346,27 @@ def main():
     # fused: score with row cuts 1, scan 1, fill 1, attention 1
     # grouped: score 1, select 4 (count, group count, scan, group fill), attention 1
     launches_per_step = 6 if a.group_select else (4 if a.fused_select else 5)
-    for _ in range(a.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    if xa.xattn_get_device_error() != xa.XATTN_OK:
-        raise RuntimeError("device error during warm-up")
+    clk = ClockSampler(local).__enter__()      # started early: nvidia-smi is slow to start
+    try:
+        for _ in range(a.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        if xa.xattn_get_device_error() != xa.XATTN_OK:
+            raise RuntimeError("device error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        clk.mark_start()
         t0.record(stream)
         for i in range(a.steps):
             step(evs[i])
         t1.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
+    finally:
+        clk.__exit__(None, None, None)
     barrier()
     total_ms = max_over_ranks(t0.elapsed_time(t1))
     ms_step = total_ms / a.steps

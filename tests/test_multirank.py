@@ -53,3 +53,19 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     w = sy.workload("tiny_1h_2k")
     assert bench.reference_arm(A, w, rank=1, world=2) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_clock_sampler_keeps_only_the_timed_window():
+    import bench
+    clk = bench.ClockSampler(0)
+    row = lambda mhz, cap: ["0", str(mhz), "1965", "700", "x", "Not Active", "Not Active",
+                            "Not Active", cap]
+    clk.rows = [(1.0, row(1965, "Not Active")),    # warm-up, before the window
+                (2.0, row(1500, "Active")),
+                (2.5, row(1520, "Active")),
+                (9.0, row(1965, "Not Active"))]    # after the window
+    clk.t_start, clk.t_end = 1.5, 2.6
+    s = clk.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1510.0 and s["reasons"] == ["sw_power_cap"]
+    clk.t_start, clk.t_end = 3.0, 3.1
+    assert clk.summary()["reasons"] == ["unsampled"]
