@@ -253,7 +253,11 @@ XATTN_API int xattn_select_noalloc(const float* scores, const float* tau, int B,
  *
  *   Q, O       bf16 [B, Hq, M, C];  K, V  bf16 [B, Hkv, M, C]
  *   row_ptr, col_idx  CSR as produced by xattn_select (device memory). Entries
- *              outside [0, M/block), and entries c > r when causal, are skipped.
+ *              outside [0, M/block), and entries c > r when causal, are skipped;
+ *              any order is accepted. The caller guarantees that every
+ *              row_ptr[i] .. row_ptr[i+1] range lies inside col_idx (the
+ *              kernel reads col_idx there without a bound; a row with
+ *              row_ptr[i+1] <= row_ptr[i] is empty).
  *   lse        fp32 [B, Hq, M] natural-log log-sum-exp of each query row's
  *              logits, or NULL. A row with no visible key gets O = 0 and
  *              lse = -inf.
