@@ -123,3 +123,27 @@ def test_full_size_sampled_rows(name, stride):
         for i, r in enumerate(rows):
             P.assert_outputs_close(got2[0, h, r * 128:(r + 1) * 128], o[i * 128:(i + 1) * 128],
                                    f"{name} O (oracle mask) h{h} r{r}")
+
+
+@pytest.mark.parametrize("name", ["llama8b_gqa_128k", "video_dit_118k"])
+def test_full_size_fused_score_select_is_bit_identical(name):
+    """The fused score+select entry point at full size: scores and kept lists
+    bit-identical to the two separate calls the bench times."""
+    w = sy.workload(name)
+    Qb, Kb, _ = sy.layer_inputs(w)
+    Q, K = to_dev(Qb), to_dev(Kb)
+    tau = torch.from_numpy(sy.tau_vector(w)).cuda()
+    ss = xa.default_score_scale(w.stride, w.C)
+    a = xa.Buffers.allocate(w.B, w.Hq, w.M, w.C, w.stride, w.causal)
+    xa.xattn_score(Q, K, w.stride, w.causal, ss, a.scores, a.score_ws)
+    xa.xattn_select(a.scores, tau, w.causal, a.row_ptr, a.col_idx, a.nnz, a.select_ws)
+    f = xa.Buffers.allocate(w.B, w.Hq, w.M, w.C, w.stride, w.causal)
+    xa.xattn_score_select(Q, K, tau, xa.XATTN_SELECT_THRESHOLD, w.stride, w.causal, ss, f.scores,
+                          f.row_ptr, f.col_idx, f.nnz, f.score_ws)
+    torch.cuda.synchronize()
+    assert xa.xattn_get_device_error() == xa.XATTN_OK
+    n = int(a.nnz.item())
+    assert int(f.nnz.item()) == n
+    assert torch.equal(a.scores, f.scores)
+    assert torch.equal(a.row_ptr, f.row_ptr)
+    assert torch.equal(a.col_idx[:n], f.col_idx[:n])
