@@ -429,6 +429,7 @@ def main():
         dense_ms = max_over_ranks(d0.elapsed_time(d1)) / a.steps
         extra["dense_attn_ms"] = dense_ms
         extra["dense_attn_tflops"] = dense_eq_flops / (dense_ms * 1e-3) / 1e12
+        extra["dense_attn_frac_of_bf16_peak"] = extra["dense_attn_tflops"] / pk["bf16_sustained"]
         extra["speedup_vs_dense"] = dense_ms / ms_step
         del Od
 
