@@ -228,3 +228,24 @@ def test_group_attention_matches_oracle(M, C, Hq, Hkv, causal):
     for h in range(Hq):
         P.assert_outputs_close(got[0, h], ref[(0, h)][0], f"O head {h}")
         np.testing.assert_allclose(glse[0, h], ref[(0, h)][1], rtol=1e-4, atol=1e-4)
+
+
+def test_group_selection_capacity_error_is_reported():
+    """A col_idx too small for the shared lists: nnz written, every list
+    withdrawn (row_ptr zero), nothing written to col_idx, ECAPACITY raised."""
+    B, Hq, Hkv, nb = 1, 4, 2, 24
+    s = np.tril(np.ones((B, Hq, nb, nb), np.float32))
+    s /= s.sum(-1, keepdims=True)
+    sc = torch.from_numpy(s).cuda()
+    pr = torch.ones(Hq, dtype=torch.float32, device="cuda")
+    row_ptr = torch.empty(B * Hkv * nb + 1, dtype=torch.int32, device="cuda")
+    col = torch.full((10,), -7, dtype=torch.int32, device="cuda")
+    nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(xa.xattn_select_group_workspace_size(B, Hq, Hkv, nb), dtype=torch.uint8,
+                     device="cuda")
+    xa.xattn_select_group(sc, pr, xa.XATTN_SELECT_THRESHOLD, Hkv, True, row_ptr, col, nnz, ws)
+    torch.cuda.synchronize()
+    assert int(nnz.item()) == B * Hkv * nb * (nb + 1) // 2
+    assert (row_ptr == 0).all() and (col == -7).all()
+    assert xa.xattn_get_device_error() == xa.XATTN_ECAPACITY
+    assert xa.xattn_get_device_error() == xa.XATTN_OK
