@@ -48,10 +48,10 @@
 namespace xattn {
 
 constexpr int kAttnTcThreads = 384;
-#ifndef XATTN_EXP2_EMU_PER4
-#define XATTN_EXP2_EMU_PER4 2
+#ifndef XATTN_EXP2_EMU_PER8
+#define XATTN_EXP2_EMU_PER8 2
 #endif
-constexpr int kEmuPer4 = XATTN_EXP2_EMU_PER4;   // softmax pairs (of 4) on the FMA pipe
+constexpr int kEmuPer8 = XATTN_EXP2_EMU_PER8;   // softmax pairs (of 8) on the FMA pipe
 // growth (log2 units) of a row's logits over its reference that one pass accepts:
 // P stays below 2^24, the row sum below 2^42 at 256K keys
 constexpr float kRefHeadroom = 24.f;
@@ -349,14 +349,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
         // the exponentials do not depend on this block's maximum, which only
-        // checks the headroom, so the two run side by side; kEmuPer4 of every 4
+        // checks the headroom, so the two run side by side; kEmuPer8 of every 8
         // pairs take the FMA-pipe exponential, the rest MUFU, so that neither
         // unit alone sets the pace of the block
 #pragma unroll
         for (int i = 0; i < 64; i += 2) {
           if (i >= 16) pm[(i >> 1) & 7] = fmax3(pm[(i >> 1) & 7], s[i], s[i + 1]);
           const float2 x = ffma2(make_float2(s[i], s[i + 1]), sc2, nm2);
-          if (((i >> 1) & 3) < kEmuPer4) {
+          if (((i >> 1) & 7) < kEmuPer8) {
             const float2 e = ex2_poly2(x);
             s[i] = e.x;
             s[i + 1] = e.y;
