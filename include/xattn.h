@@ -249,7 +249,11 @@ XATTN_API int xattn_select_noalloc(const float* scores, const float* tau, int B,
  * For query token i of block r of head h (KV head h/(Hq/Hkv)):
  *   O[i] = sum_j softmax_j(softmax_scale * q_i . k_j) v_j
  * over the tokens j of the kept key blocks of row (b,h,r) (and j <= i when
- * causal). Accumulation and softmax are fp32; O is rounded to bf16.
+ * causal). Accumulation and softmax are fp32; O is rounded to bf16. The
+ * unnormalised weights are taken against one reference per row (its first kept
+ * block's maximum; a tile whose logits outgrow it by more than 2^24 is computed
+ * again against the true maximum), so they stay below 2^24 and the fp32
+ * accumulators stay finite for |V| < 2^86.
  *
  *   Q, O       bf16 [B, Hq, M, C];  K, V  bf16 [B, Hkv, M, C]
  *   row_ptr, col_idx  CSR as produced by xattn_select (device memory). Entries
