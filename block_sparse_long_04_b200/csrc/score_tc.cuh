@@ -15,9 +15,11 @@
 // tcgen05 MMAs into a TMEM accumulator, double-buffered so that the epilogue of
 // one column tile overlaps the MMAs of the next.
 //
-// Warp roles (256 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA
-// issuer (warp 1 also owns the TMEM allocation), warps 4-7 = epilogue, one
-// reshaped row per thread (TMEM lane = row); all eight warps share the finalize.
+// Warp roles (384 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA
+// issuer (warp 1 also owns the TMEM allocation), warps 4-11 = epilogue, two
+// threads per reshaped row (TMEM lane = row): warps 4-7 take the first half of
+// every column tile, warps 8-11 the second, each with its own running row LSE,
+// merged once at the end; all twelve warps share the finalize.
 //
 // Epilogue (row softmax + block summation, XAttention summary, Approach): for
 // every key block of g = 128/S columns the thread forms the block's base-2
@@ -38,7 +40,7 @@
 
 namespace xattn {
 
-constexpr int kScoreTcThreads = 256;
+constexpr int kScoreTcThreads = 384;
 
 template <int BN>
 struct ScoreTc {
@@ -48,7 +50,8 @@ struct ScoreTc {
   static constexpr int kStageBytes = kQBytes + kKBytes;
   static constexpr int kOffBar = kStages * kStageBytes;
   static constexpr int kOffLse = kOffBar + 256;
-  static constexpr int kSmem = kOffLse + 128 * 4 + 16 + 1024;
+  static constexpr int kOffX = kOffLse + 128 * 4 + 16;   // [2 halves][128] (max, sum)
+  static constexpr int kSmem = kOffX + 2 * 128 * 8 + 1024;
   static constexpr int kTmemCols = 2 * BN;
 };
 
@@ -86,6 +89,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* lse_s = reinterpret_cast<float*>(smem + L::kOffLse);
+  float2* xchg = reinterpret_cast<float2*>(smem + L::kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rp = M / S;
@@ -101,7 +105,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (tid == 0) {
     for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -169,6 +173,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else if (warp >= 4) {
     // -------------------------------------------------------------- epilogue
+    static_assert(BN == 256, "two epilogue threads per row take 128 columns each");
+    constexpr int CH = G > 64 ? 128 : 64;      // columns per TMEM read (whole blocks)
+    const int hh = (warp - 4) >> 2;            // column half of every tile
     const int rl = (warp & 3) * 32 + lane;     // row within the tile
     const int ip = i0 + rl;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -180,20 +187,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int half = 0; half < BN / 128; ++half) {
-        float v[128];
+      for (int ch = 0; ch < 128 / CH; ++ch) {
+        float v[CH];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          tmem_ld32(tmem + lane_off + buf * BN + half * 128 + q4 * 32, v + q4 * 32);
+        for (int q4 = 0; q4 < CH / 32; ++q4)
+          tmem_ld32(tmem + lane_off + buf * BN + hh * 128 + ch * CH + q4 * 32, v + q4 * 32);
         tmem_wait_ld();
-        if (half == BN / 128 - 1) {
+        if (ch == 128 / CH - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
-        const int j0 = jt * BN + half * 128;
+        const int j0 = jt * BN + hh * 128 + ch * CH;
 #pragma unroll
-        for (int kb = 0; kb < 128 / G; ++kb) {
+        for (int kb = 0; kb < CH / G; ++kb) {
           float vmax = kNegInf;
 #pragma unroll
           for (int i = 0; i < G; ++i) {
@@ -217,19 +224,28 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
 
-    // ---- row LSE, then the finalize by all warps ----
-    if (ok) {
-      const float L_row = (l_run > 0.f) ? m_run + lg2(l_run) : kNegInf;
+    // ---- row LSE from the two halves, then the finalize by all warps ----
+    xchg[hh * 128 + rl] = make_float2(m_run, l_run);
+    asm volatile("bar.sync 3, 256;" ::: "memory");
+    if (hh == 0 && !*abort_flag) {
+      const float2 o = xchg[128 + rl];
+      const float mm = fmaxf(m_run, o.x);
+      float lt = 0.f;
+      if (mm != kNegInf) {
+        if (m_run != kNegInf) lt += l_run * ex2(m_run - mm);
+        if (o.x != kNegInf) lt += o.y * ex2(o.x - mm);
+      }
+      const float L_row = (lt > 0.f) ? mm + lg2(lt) : kNegInf;
       lse_s[rl] = L_row;
       if (ip < rp) lse_ws[(size_t)bh * rp + ip] = L_row;
     }
     tc_fence_before();
   }
 
-  // The producer and MMA warps are idle by now, so all 256 threads turn the
+  // The producer and MMA warps are idle by now, so all 384 threads turn the
   // partials of the CTA's rows into block scores (a wait that failed has set
   // the abort flag, which every thread reads after the barrier).
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+  asm volatile("bar.sync 1, 384;" ::: "memory");
   const bool done_ok = !*abort_flag;
   if (done_ok) {
     const float inv_g = 1.f / (float)G;
@@ -251,9 +267,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   }
   if (SELECT) {
-    // fused selection of the rows just written, by the 128 epilogue threads
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (warp >= 4) {
+    // fused selection of the rows just written, by the 128 threads of warps 4-7
+    asm volatile("bar.sync 1, 384;" ::: "memory");
+    if (warp >= 4 && warp < 8) {
       const int et = tid - 128;
       if (done_ok) {
         uint64_t* keys = reinterpret_cast<uint64_t*>(smem);             // the idle stage ring
