@@ -35,6 +35,12 @@ sys.path.insert(0, ROOT)
 import synthetic as sy  # noqa: E402
 
 METRIC = "128K-token prefill attention ms/layer and kept-block TFLOPS (% of BF16 peak)"
+# scale of the scoring softmax (name -> (description, value for stride S and head dim C))
+SCORE_SCALES = {
+    "sqrt_sc": ("1/sqrt(stride*C)", lambda S, C: 1.0 / math.sqrt(S * C)),
+    "sqrt_c": ("1/sqrt(C)", lambda S, C: 1.0 / math.sqrt(C)),
+    "s_sqrt_c": ("1/(stride*sqrt(C))", lambda S, C: 1.0 / (S * math.sqrt(C))),
+}
 UNIT = "ms/layer"
 
 
@@ -54,6 +60,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fused-select", action="store_true",
                     help="score and select in the one fused call instead of two calls")
+    ap.add_argument("--score-scale", default="sqrt_sc", choices=sorted(SCORE_SCALES),
+                    help="scale of the scoring softmax: 1/sqrt(stride*C) (default), "
+                         "1/sqrt(C) or 1/(stride*sqrt(C)); the method leaves it open")
     ap.add_argument("--group-select", action="store_true",
                     help="GQA-shared kept lists (union over each KV group; a variant the "
                          "method does not define) instead of per-head lists")
@@ -168,14 +177,18 @@ class ClockSampler:
 
 
 # --------------------------------------------------------- CPU oracle sample
-def oracle_sample(w, Qb, Kb, Vb, tau, seconds, seed=0):
+def score_scale_of(a, w) -> float:
+    return SCORE_SCALES[a.score_scale][1](w.stride, w.C)
+
+
+def oracle_sample(w, Qb, Kb, Vb, tau, seconds, sig, seed=0):
     """Time the oracle on uniformly drawn (head, query block) units until `seconds`
     of work are done; returns (ms per layer extrapolated by unit count, units, desc)."""
     import oracle as orc
     from threadpoolctl import threadpool_info
     rng = np.random.default_rng(seed)
     nb, grp = w.nb, w.Hq // w.Hkv
-    sig, sa = orc.default_score_scale(w.stride, w.C), 1 / math.sqrt(w.C)
+    sa = 1 / math.sqrt(w.C)
     done, t_work = 0, 0.0
     cache = {}
     while t_work < seconds or done < 4:
@@ -206,10 +219,11 @@ def reference_arm(a, w, rank, world):
     tau = sy.tau_vector(w, a.seed)
     per_step = max(2.0, min(a.cpu_seconds, 60.0 / max(1, a.steps + a.warmup)))
     for i in range(a.warmup):
-        oracle_sample(w, Qb, Kb, Vb, tau, per_step, seed=100 + i)
+        oracle_sample(w, Qb, Kb, Vb, tau, per_step, score_scale_of(a, w), seed=100 + i)
     vals, units, cores, desc = [], 0, 1, ""
     for i in range(a.steps):
-        v, u, desc, cores = oracle_sample(w, Qb, Kb, Vb, tau, per_step, seed=i)
+        v, u, desc, cores = oracle_sample(w, Qb, Kb, Vb, tau, per_step, score_scale_of(a, w),
+                                          seed=i)
         vals.append(v)
         units += u
     val = statistics.mean(vals)
@@ -217,7 +231,7 @@ def reference_arm(a, w, rank, world):
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": val, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w),
+        "config": config_of(w, a),
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"per step: {desc}"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -226,11 +240,11 @@ def reference_arm(a, w, rank, world):
     return 0
 
 
-def config_of(w):
+def config_of(w, a):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.M, "C": w.C,
             "block": w.block, "stride": w.stride, "causal": w.causal,
             "tau": list(w.tau_range) if w.tau_range else w.tau,
-            "score_scale": "1/sqrt(stride*C)", "softmax_scale": "1/sqrt(C)",
+            "score_scale": SCORE_SCALES[a.score_scale][0], "softmax_scale": "1/sqrt(C)",
             "l2": "no flush; inputs larger than L2 (126 MB): Q %.2f GB, K and V %.2f GB each" % (
                 w.B * w.Hq * w.M * w.C * 2 / 1e9, w.B * w.Hkv * w.M * w.C * 2 / 1e9)
             if w.B * w.Hkv * w.M * w.C * 2 > 126e6 else "inputs fit in L2 (not a bench workload)",
@@ -294,7 +308,7 @@ def main():
     tau = torch.from_numpy(tau_np).to(dev)
     bufs = xa.Buffers.allocate(w.B, w.Hq, w.M, w.C, w.stride, w.causal, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ss = xa.default_score_scale(w.stride, w.C)
+    ss = score_scale_of(a, w)
     sa = 1 / math.sqrt(w.C)
 
     G = w.Hq // w.Hkv
@@ -464,7 +478,8 @@ def main():
                 stream.wait_event(h2d_done[sb])
                 if i >= 2:                       # O of step i-2 has been copied out
                     stream.wait_event(d2h_done[sb])
-                xa.xattn_prefill(q, k, v, t, w.stride, w.causal, bb, stream=stream)
+                xa.xattn_prefill(q, k, v, t, w.stride, w.causal, bb, score_scale=ss,
+                                 stream=stream)
                 comp_done[sb].record(stream)
                 d2h.wait_event(comp_done[sb])
                 with torch.cuda.stream(d2h):
@@ -493,14 +508,14 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        v, units, desc, cores = oracle_sample(w, *views, tau_np, a.cpu_seconds)
+        v, units, desc, cores = oracle_sample(w, *views, tau_np, a.cpu_seconds, ss)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(config_of(w), selection=(
+        "config": dict(config_of(w, a), selection=(
             "GQA-shared union over each KV group (variant)" if a.group_select else
             "per head, fused with scoring" if a.fused_select else "per head")),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,

@@ -1,6 +1,8 @@
 """The multi-rank host logic of bench.py on CPU (gloo, world size 2): the job time
 is the max over ranks, the whole-job metric divides by every rank's layers, and
 the reference arm runs on rank 0 only."""
+import json
+import math
 import os
 import socket
 
@@ -53,6 +55,23 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     w = sy.workload("tiny_1h_2k")
     assert bench.reference_arm(A, w, rank=1, world=2) == 0
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("name,desc", [("sqrt_sc", "1/sqrt(stride*C)"), ("sqrt_c", "1/sqrt(C)"),
+                                       ("s_sqrt_c", "1/(stride*sqrt(C))")])
+def test_reference_arm_reports_the_score_scale(capsys, name, desc):
+    """The scoring-softmax scale the method leaves open is a bench option; the
+    reference line names the one it timed the oracle with."""
+    class A:
+        seed, steps, warmup, cpu_seconds, gpus, score_scale = 1, 1, 0, 0.05, 1, name
+    w = sy.workload("tiny_1h_2k")
+    assert bench.reference_arm(A, w, rank=0, world=1) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["score_scale"] == desc
+    S, C = w.stride, w.C
+    want = {"sqrt_sc": 1 / math.sqrt(S * C), "sqrt_c": 1 / math.sqrt(C),
+            "s_sqrt_c": 1 / (S * math.sqrt(C))}[name]
+    assert math.isclose(bench.score_scale_of(A, w), want)
 
 
 def test_clock_sampler_keeps_only_the_timed_window():
