@@ -268,34 +268,27 @@ size_t xattn_select_workspace_size(int B, int Hq, int nb) {
   return (bytes + 255) & ~(size_t)255;
 }
 
-static int select_common(const float* scores, const float* param, int rule, int B, int Hq, int nb,
+// Checks and launches of the per-head selection (count, scan, fill) with the
+// per-row scratch `cuts` supplied by the caller of this helper: the workspace of
+// xattn_select / xattn_select_ex, or the library's fixed array for
+// xattn_select_noalloc. `cuts` may be null only when there are no rows.
+static int select_launch(const float* scores, const float* param, int rule, int B, int Hq, int nb,
                          int causal, int32_t* row_ptr, int32_t* col_idx, size_t col_capacity,
-                         int32_t* nnz, void* workspace, size_t workspace_bytes, void* stream) {
-  if (B < 0 || Hq < 0 || nb < 0) return XATTN_EINVAL;
-  if (rule != kSelThreshold && rule != kSelTopK && rule != kSelRatio) return XATTN_EINVAL;
+                         int32_t* nnz, SelCut* cuts, cudaStream_t st) {
   const long long rows = (long long)B * Hq * nb;
-  if (nb > kSelMaxNb) return XATTN_EUNSUPPORTED;
-  // worst-case kept entries must fit the int32 row_ptr
-  const long long worst = causal ? rows * (nb + 1) / 2 : rows * nb;
-  if (worst >= (1LL << 31) || rows >= (1LL << 31) - 1) return XATTN_EUNSUPPORTED;
-  if (!row_ptr || !nnz) return XATTN_EINVAL;
-  cudaStream_t st = as_stream(stream);
   if (rows == 0) {
     // nothing to select: row_ptr = {0}, nnz = 0
     if (cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
     if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
     return XATTN_OK;
   }
-  if (!scores || !param || !col_idx || !workspace) return XATTN_EINVAL;
-  if (workspace_bytes < xattn_select_workspace_size(B, Hq, nb)) return XATTN_EINVAL;
-  if (((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
-  SelCut* cuts = static_cast<SelCut*>(workspace);
+  if (!scores || !param || !col_idx) return XATTN_EINVAL;
+  if (cuts == nullptr) return XATTN_ECUDA;
   int P = 1;
   while (P < nb) P <<= 1;
-  const int smem = P * 8;
   static unsigned long long done = 0;
   if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
-  select_count_kernel<<<(unsigned)rows, kSelThreads, smem, st>>>(scores, param, Hq, nb,
+  select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, param, Hq, nb,
                                                                   causal ? 1 : 0, cuts, rule);
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
   const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
@@ -304,6 +297,34 @@ static int select_common(const float* scores, const float* param, int rule, int 
   select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
                                                               row_ptr, col_idx);
   return launch_status();
+}
+
+// Shape and rule checks shared by every per-head selection entry point.
+static int select_check(int rule, int B, int Hq, int nb, int causal, const int32_t* row_ptr,
+                        const int32_t* nnz) {
+  if (B < 0 || Hq < 0 || nb < 0) return XATTN_EINVAL;
+  if (rule != kSelThreshold && rule != kSelTopK && rule != kSelRatio) return XATTN_EINVAL;
+  const long long rows = (long long)B * Hq * nb;
+  if (nb > kSelMaxNb) return XATTN_EUNSUPPORTED;
+  // worst-case kept entries must fit the int32 row_ptr
+  const long long worst = causal ? rows * (nb + 1) / 2 : rows * nb;
+  if (worst >= (1LL << 31) || rows >= (1LL << 31) - 1) return XATTN_EUNSUPPORTED;
+  if (!row_ptr || !nnz) return XATTN_EINVAL;
+  return XATTN_OK;
+}
+
+static int select_common(const float* scores, const float* param, int rule, int B, int Hq, int nb,
+                         int causal, int32_t* row_ptr, int32_t* col_idx, size_t col_capacity,
+                         int32_t* nnz, void* workspace, size_t workspace_bytes, void* stream) {
+  const int rc = select_check(rule, B, Hq, nb, causal, row_ptr, nnz);
+  if (rc != XATTN_OK) return rc;
+  if ((long long)B * Hq * nb > 0) {
+    if (!workspace) return XATTN_EINVAL;
+    if (workspace_bytes < xattn_select_workspace_size(B, Hq, nb)) return XATTN_EINVAL;
+    if (((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
+  }
+  return select_launch(scores, param, rule, B, Hq, nb, causal, row_ptr, col_idx, col_capacity,
+                       nnz, static_cast<SelCut*>(workspace), as_stream(stream));
 }
 
 int xattn_select(const float* scores, const float* tau, int B, int Hq, int nb, int causal,
@@ -443,34 +464,17 @@ int xattn_select_noalloc(const float* scores, const float* tau, int B, int Hq, i
                          int32_t* row_ptr, int32_t* col_idx, size_t col_capacity, int32_t* nnz,
                          void* stream) {
   if (B < 0 || Hq < 0 || nb < 0) return XATTN_EINVAL;
-  const long long rows = (long long)B * Hq * nb;
-  if (nb > kSelMaxNb || rows > XATTN_SELECT_NOALLOC_MAX_ROWS) return XATTN_EUNSUPPORTED;
-  const long long worst = causal ? rows * (nb + 1) / 2 : rows * nb;
-  if (worst >= (1LL << 31)) return XATTN_EUNSUPPORTED;
-  if (!row_ptr || !nnz) return XATTN_EINVAL;
-  cudaStream_t st = as_stream(stream);
-  if (rows == 0) {
-    if (cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
-    if (cudaMemsetAsync(nnz, 0, sizeof(int32_t), st) != cudaSuccess) return XATTN_ECUDA;
-    return XATTN_OK;
+  if ((long long)B * Hq * nb > XATTN_SELECT_NOALLOC_MAX_ROWS) return XATTN_EUNSUPPORTED;
+  const int rc = select_check(kSelThreshold, B, Hq, nb, causal, row_ptr, nnz);
+  if (rc != XATTN_OK) return rc;
+  SelCut* cuts = nullptr;
+  if ((long long)B * Hq * nb > 0) {
+    if (!scores || !tau || !col_idx) return XATTN_EINVAL;
+    cuts = select_scratch_on_current_device();
+    if (cuts == nullptr) return XATTN_ECUDA;
   }
-  if (!scores || !tau || !col_idx) return XATTN_EINVAL;
-  SelCut* cuts = select_scratch_on_current_device();
-  if (cuts == nullptr) return XATTN_ECUDA;
-  int P = 1;
-  while (P < nb) P <<= 1;
-  static unsigned long long done = 0;
-  if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
-  select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, tau, Hq, nb,
-                                                                  causal ? 1 : 0, cuts,
-                                                                  kSelThreshold);
-  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
-  const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
-  select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
-  if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
-  select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
-                                                              row_ptr, col_idx);
-  return launch_status();
+  return select_launch(scores, tau, kSelThreshold, B, Hq, nb, causal, row_ptr, col_idx,
+                       col_capacity, nnz, cuts, as_stream(stream));
 }
 
 int xattn_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* row_ptr,

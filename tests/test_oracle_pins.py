@@ -414,3 +414,93 @@ def test_layer_group_maps_heads_to_their_kv_head():
     kept[(0, 2)][1] = np.array([1])
     kept[(0, 3)][1] = np.array([1])
     assert orc.layer_select_group(kept, Hq=4, Hkv=2)[(0, 1)][1].tolist() == [1]
+
+
+# ------------------------------------------------ layer wrappers (GQA, per-head tau)
+# Query head -> KV head for Hq = 4 query heads sharing Hkv = 2 KV heads, written out
+# by hand: heads 0 and 1 read KV head 0, heads 2 and 3 read KV head 1 (the GQA head
+# sharing of the Llama-shaped workloads; each query head keeps its own threshold,
+# XAttention summary, "Approach").
+_GQA_KV_OF = {0: 0, 1: 0, 2: 1, 3: 1}
+_GQA_TAU = np.array([0.35, 0.6, 0.85, 0.97])
+
+
+def _gqa_layer(seed=21, B=2, M=96, C=8):
+    import synthetic as sy
+    rng = np.random.default_rng(seed)
+    # KV heads differ strongly (their own scale and offset), so a wrong head mapping
+    # moves every score, kept list and output
+    Q = rng.standard_normal((B, 4, M, C)).astype(np.float32)
+    K = rng.standard_normal((B, 2, M, C)).astype(np.float32)
+    V = rng.standard_normal((B, 2, M, C)).astype(np.float32)
+    K[:, 1] = 2.5 * K[:, 1] + 1.0
+    V[:, 1] = V[:, 1] - 3.0
+    return sy.bf16_round(Q), sy.bf16_round(K), sy.bf16_round(V)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_layer_wrappers_map_query_heads_and_taus(causal):
+    """layer_block_scores / layer_select / layer_sparse_attention on a B = 2,
+    Hq = 4, Hkv = 2 layer equal the single-head functions called on hand-sliced
+    (q of head h, k and v of KV head _GQA_KV_OF[h]) with that head's own tau."""
+    S, b = 4, 16
+    Qb, Kb, Vb = _gqa_layer()
+    B = Qb.shape[0]
+    sig, sa = 0.3, 0.25
+    scores = orc.layer_block_scores(Qb, Kb, 2, S, b, sig, causal)
+    kept = orc.layer_select(scores, _GQA_TAU, causal)
+    outs = orc.layer_sparse_attention(Qb, Kb, Vb, 2, kept, b, causal, sa)
+    assert sorted(scores) == [(bb, h) for bb in range(B) for h in range(4)]
+    for bb in range(B):
+        for h in range(4):
+            kv = _GQA_KV_OF[h]
+            q = orc.bf16_to_f64(Qb[bb, h])
+            k = orc.bf16_to_f64(Kb[bb, kv])
+            v = orc.bf16_to_f64(Vb[bb, kv])
+            want_s = orc.block_scores(q, k, S, b, sig, causal)
+            np.testing.assert_array_equal(scores[(bb, h)], want_s)
+            want_k = orc.select_blocks(want_s, float(_GQA_TAU[h]), causal)
+            assert {r: x.tolist() for r, x in kept[(bb, h)].items()} == \
+                {r: x.tolist() for r, x in want_k.items()}
+            want_o, want_l = orc.block_sparse_attention(q, k, v, want_k, b, causal, sa)
+            np.testing.assert_array_equal(outs[(bb, h)][0], want_o)
+            np.testing.assert_array_equal(outs[(bb, h)][1], want_l)
+
+
+def _wrong_kv_mapping(Qb, Kb, Hkv, stride, block, sigma, causal, heads=None, rows=None,
+                      antidiagonal=True):
+    """A plausible slip: query head h read KV head h % Hkv instead of its group's."""
+    B, Hq = Qb.shape[:2]
+    heads = [(bb, h) for bb in range(B) for h in range(Hq)] if heads is None else heads
+    return {(bb, h): orc.block_scores(orc.bf16_to_f64(Qb[bb, h]), orc.bf16_to_f64(Kb[bb, h % Hkv]),
+                                      stride, block, sigma, causal, rows, antidiagonal)
+            for (bb, h) in heads}
+
+
+def test_planted_wrong_kv_head_mapping_is_caught(monkeypatch):
+    monkeypatch.setattr(orc, "layer_block_scores", _wrong_kv_mapping)
+    with pytest.raises(AssertionError):
+        test_layer_wrappers_map_query_heads_and_taus(True)
+
+
+def test_planted_group_tau_is_caught(monkeypatch):
+    """A plausible slip: every head of a group used the group's tau[h // grp]."""
+    def wrong(scores_by_head, tau, causal, rows=None):
+        return {(bb, h): orc.select_blocks(s, float(tau[h // 2]), causal, rows)
+                for (bb, h), s in scores_by_head.items()}
+    monkeypatch.setattr(orc, "layer_select", wrong)
+    with pytest.raises(AssertionError):
+        test_layer_wrappers_map_query_heads_and_taus(True)
+
+
+def test_planted_wrong_attention_kv_head_is_caught(monkeypatch):
+    """A plausible slip in the attention wrapper: V taken from KV head h % Hkv."""
+    def wrong(Qb, Kb, Vb, Hkv, kept_by_head, block, causal, scale, rows=None):
+        grp = Qb.shape[1] // Hkv
+        return {(bb, h): orc.block_sparse_attention(
+            orc.bf16_to_f64(Qb[bb, h]), orc.bf16_to_f64(Kb[bb, h // grp]),
+            orc.bf16_to_f64(Vb[bb, h % Hkv]), kept, block, causal, scale, rows)
+            for (bb, h), kept in kept_by_head.items()}
+    monkeypatch.setattr(orc, "layer_sparse_attention", wrong)
+    with pytest.raises(AssertionError):
+        test_layer_wrappers_map_query_heads_and_taus(False)

@@ -8,8 +8,9 @@ library. Its kept lists must equal those of xattn_select exactly (they are
 integer outputs), call after call, although every call reuses the same scratch.
 
 This file is collected last, so that a run stopping at its first failure has
-already run every other test; it sets up everything it needs itself, so it also
-passes when run alone in a fresh process.
+already run every other test. It builds the library itself (a no-op when the
+build is current) and sets up every input it needs, so it also passes when run
+alone in a fresh process.
 """
 import ctypes
 
@@ -17,7 +18,10 @@ import numpy as np
 import pytest
 import torch
 
-import block_sparse_long_04_b200 as xa
+from block_sparse_long_04_b200 import build as _build
+
+_build.build()
+import block_sparse_long_04_b200 as xa  # noqa: E402
 
 
 def _scores(seed, Hq, nb, causal):
@@ -68,10 +72,53 @@ def test_noalloc_select_equals_select_on_consecutive_calls():
         assert torch.equal(ci[:n], ref[1][:n])
 
 
+def _call(ptrs, B, Hq, nb, causal, cap, stream=None):
+    sc, tau, rp, ci, nz = (ctypes.c_void_p(p) if p is not None else None for p in ptrs)
+    return xa._lib.xattn_select_noalloc(sc, tau, B, Hq, nb, int(causal), rp, ci, cap, nz, stream)
+
+
 def test_noalloc_select_rejects_rows_beyond_its_scratch():
     # checked on the host before any launch: no GPU needed
-    fake = ctypes.c_void_p(0x7F0000001000)
-    nb = 2048
-    Hq = xa.XATTN_SELECT_NOALLOC_MAX_ROWS // nb + 1
-    rc = xa._lib.xattn_select_noalloc(fake, fake, 1, Hq, nb, 1, fake, fake, 1 << 30, fake, None)
-    assert rc == xa.XATTN_EUNSUPPORTED
+    fake = 0x7F0000001000
+    top = xa.XATTN_SELECT_NOALLOC_MAX_ROWS
+    # one row beyond the scratch array
+    assert _call([fake] * 5, 1, top + 1, 1, True, 1 << 30) == xa.XATTN_EUNSUPPORTED
+    assert _call([fake] * 5, 1, top // 2048 + 1, 2048, True, 1 << 30) == xa.XATTN_EUNSUPPORTED
+    # exactly the scratch size passes the size check: with no output pointers the
+    # call then stops at the argument check, still before any launch
+    assert _call([fake, fake, None, fake, None], 1, top, 1, True, 1 << 30) == xa.XATTN_EINVAL
+    assert _call([fake, fake, None, fake, None], 2, top // 2048, 1024, True,
+                 1 << 30) == xa.XATTN_EINVAL
+
+
+@pytest.mark.gpu
+def test_noalloc_select_fills_its_whole_scratch():
+    """Exactly XATTN_SELECT_NOALLOC_MAX_ROWS rows (B = 2, 128 heads, 1024 query
+    blocks), so the last row lands in the last slot of the fixed array; the kept
+    lists must equal xattn_select's."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    B, Hq, nb, causal = 2, 128, 1024, True
+    assert B * Hq * nb == xa.XATTN_SELECT_NOALLOC_MAX_ROWS
+    g = torch.Generator(device="cuda").manual_seed(7)
+    s = torch.rand((B, Hq, nb, nb), device="cuda", generator=g) ** 6
+    s = torch.tril(s)
+    s /= s.sum(dim=-1, keepdim=True)
+    tau = torch.linspace(0.5, 0.98, Hq, device="cuda")
+    cap = xa.max_kept(B, Hq, nb, causal)
+    ref = (torch.full((B * Hq * nb + 1,), -1, dtype=torch.int32, device="cuda"),
+           torch.full((cap,), -1, dtype=torch.int32, device="cuda"),
+           torch.full((1,), -1, dtype=torch.int32, device="cuda"))
+    ws = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8, device="cuda")
+    xa.xattn_select(s, tau, causal, *ref, ws)
+    got = tuple(torch.full_like(t, -1) for t in ref)
+    rc = _call([s.data_ptr(), tau.data_ptr(), got[0].data_ptr(), got[1].data_ptr(),
+                got[2].data_ptr()], B, Hq, nb, causal, cap,
+               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == xa.XATTN_OK, xa.status_string(rc)
+    torch.cuda.synchronize()
+    assert xa.xattn_get_device_error() == xa.XATTN_OK
+    n = int(ref[2].item())
+    assert int(got[2].item()) == n
+    assert torch.equal(got[0], ref[0])
+    assert torch.equal(got[1][:n], ref[1][:n])
