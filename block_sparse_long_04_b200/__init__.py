@@ -35,7 +35,7 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "xattn_status_string": (ctypes.c_char_p, [_I]),
     "xattn_version": (_I, []),
-    "xattn_score_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "xattn_score_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "xattn_score": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _Z, _P]),
     "xattn_select_workspace_size": (_Z, [_I, _I, _I]),
     "xattn_select": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
@@ -51,7 +51,7 @@ SIGNATURES = {
     "xattn_select_group": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P, _Z, _P]),
     "xattn_sparse_attn_group": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P,
                                      _P]),
-    "xattn_score_select_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "xattn_score_select_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "xattn_score_select": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _Z,
                                 _P, _P, _Z, _P]),
 }
@@ -123,8 +123,10 @@ def _bf16(*ts):
 
 
 # ------------------------------------------------------------------ sizes
-def xattn_score_workspace_size(B: int, Hq: int, M: int, stride: int, block: int = 128) -> int:
-    return int(_lib.xattn_score_workspace_size(B, Hq, M, stride, block))
+def xattn_score_workspace_size(B: int, Hq: int, M: int, stride: int, causal: bool,
+                               block: int = 128) -> int:
+    """Bytes of the scoring workspace; sized for the `causal` flag of the call."""
+    return int(_lib.xattn_score_workspace_size(B, Hq, M, stride, block, int(causal)))
 
 
 def xattn_select_workspace_size(B: int, Hq: int, nb: int) -> int:
@@ -188,8 +190,9 @@ def xattn_select_group(scores, param, rule: int, Hkv: int, causal: bool, row_ptr
     _check(rc, "xattn_select_group")
 
 
-def xattn_score_select_workspace_size(B: int, Hq: int, M: int, stride: int, block: int = 128) -> int:
-    return int(_lib.xattn_score_select_workspace_size(B, Hq, M, stride, block))
+def xattn_score_select_workspace_size(B: int, Hq: int, M: int, stride: int, causal: bool,
+                                      block: int = 128) -> int:
+    return int(_lib.xattn_score_select_workspace_size(B, Hq, M, stride, block, int(causal)))
 
 
 def xattn_score_select(Q, K, param, rule: int, stride: int, causal: bool, score_scale: float, scores,
@@ -319,7 +322,8 @@ class Buffers:
         return Buffers(
             scores=torch.empty((B, Hq, nb, nb), dtype=torch.float32, device=dev),
             # sized for the fused score+select call, which also serves xattn_score
-            score_ws=torch.empty(max(1, xattn_score_select_workspace_size(B, Hq, M, stride, block)),
+            score_ws=torch.empty(max(1, xattn_score_select_workspace_size(B, Hq, M, stride, causal,
+                                                                          block)),
                                  dtype=torch.uint8, device=dev),
             select_ws=torch.empty(max(1, xattn_select_workspace_size(B, Hq, nb)),
                                   dtype=torch.uint8, device=dev),

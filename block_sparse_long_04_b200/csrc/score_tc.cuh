@@ -65,6 +65,17 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 static_assert(ScoreTc<128>::kOffBar >= kSelMaxNb * 8 + 64 && ScoreTc<256>::kOffBar >= kSelMaxNb * 8 + 64,
               "the stage ring must hold the fused selection's sort keys");
 
+// Offset of reshaped row ip's partial log-masses in the workspace. Non-causal:
+// nb entries per row. Causal: the g = G rows of query block r hold only the
+// r + 1 key blocks they can see, so head bh's rows are packed as a triangle of
+// G * nb * (nb + 1) / 2 = rp * (nb + 1) / 2 entries (half of the non-causal size).
+template <int G>
+__device__ __forceinline__ size_t part_row(int bh, int ip, int rp, int nb, int causal) {
+  if (!causal) return ((size_t)bh * rp + ip) * nb;
+  const size_t r = (size_t)(ip / G), i = (size_t)(ip % G);
+  return (size_t)bh * ((size_t)rp * (nb + 1) / 2) + G * (r * (r + 1) / 2) + i * (r + 1);
+}
+
 template <int C, int G, int BN, bool SELECT>
 __global__ void __launch_bounds__(kScoreTcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -218,7 +229,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const float mn = fmaxf(m_run, ell);
             l_run = l_run * ex2(m_run - mn) + ex2(ell - mn);
             m_run = mn;
-            if (ip < rp) part[((size_t)bh * rp + ip) * nb + (j0 / G + kb)] = ell;
+            if (ip < rp) part[part_row<G>(bh, ip, rp, nb, causal) + (j0 / G + kb)] = ell;
           }
         }
       }
@@ -254,12 +265,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (r >= nb) break;
       const int ncand = causal ? r + 1 : nb;
       float* srow = scores + ((size_t)bh * nb + r) * nb;
-      const float* pr0 = part + ((size_t)bh * rp + (size_t)r * G) * nb;
+      const float* pr0 = part + part_row<G>(bh, r * G, rp, nb, causal);
       for (int c = tid; c < nb; c += kScoreTcThreads) {
         float acc = 0.f;
         if (c < ncand) {
 #pragma unroll 4
-          for (int i = 0; i < G; ++i) acc += ex2(pr0[(size_t)i * nb + c] - lse_s[r * G + i - i0]);
+          for (int i = 0; i < G; ++i) acc += ex2(pr0[(size_t)i * ncand + c] - lse_s[r * G + i - i0]);
           acc *= inv_g;
         }
         srow[c] = acc;

@@ -83,7 +83,8 @@ bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int width,
 }
 
 bool stride_supported(int stride) {
-  return stride == 1 || stride == 2 || stride == 4 || stride == 8 || stride == 16;
+  return stride == 1 || stride == 2 || stride == 4 || stride == 8 || stride == 16 ||
+         stride == 32 || stride == 64;
 }
 
 // Shared shape checks; returns XATTN_OK, XATTN_EINVAL or XATTN_EUNSUPPORTED.
@@ -97,6 +98,13 @@ int check_shape(int B, int Hq, int Hkv, int M, int C, int block) {
   // element offsets stay below 2^62; grid dimensions below their limits
   if ((long long)B * Hq > 65535) return XATTN_EUNSUPPORTED;
   return XATTN_OK;
+}
+
+// fp32 partial log-masses of the scoring workspace: one per (reshaped row, key
+// block) it can see, i.e. rp * nb per head, or rp * (nb + 1) / 2 when causal.
+size_t score_part_entries(int B, int Hq, int M, int stride, int block, int causal) {
+  const size_t rp = (size_t)M / stride, nb = (size_t)M / block;
+  return (size_t)B * Hq * (causal ? rp * (nb + 1) / 2 : rp * nb);
 }
 
 // Optional fused selection of the scoring kernel: rule + per-head parameter, and
@@ -142,6 +150,8 @@ int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int 
     case 4: return launch_score_tc<C, 32, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
     case 8: return launch_score_tc<C, 16, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
     case 16: return launch_score_tc<C, 8, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
+    case 32: return launch_score_tc<C, 4, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
+    case 64: return launch_score_tc<C, 2, SELECT>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale, scores, part, lse_ws, fs, st);
   }
   return XATTN_EUNSUPPORTED;
 }
@@ -206,12 +216,12 @@ int score_common(const void* Q, const void* K, int B, int Hq, int Hkv, int M, in
   if (!aligned16(Q) || !aligned16(K) || !aligned16(workspace) || !aligned16(scores))
     return XATTN_EINVAL;
   if (!(score_scale > 0.f) || score_scale == __builtin_huge_valf()) return XATTN_EINVAL;
-  const size_t need = xattn_score_workspace_size(B, Hq, M, stride, block);
+  const size_t need = xattn_score_workspace_size(B, Hq, M, stride, block, causal);
   if (workspace_bytes < need) return XATTN_EINVAL;
   const int rp = M / stride;
   if ((rp + 127) / 128 > (1 << 30)) return XATTN_EUNSUPPORTED;
   float* part = static_cast<float*>(workspace);
-  float* lse_ws = part + (size_t)B * Hq * rp * (M / block);
+  float* lse_ws = part + score_part_entries(B, Hq, M, stride, block, causal);
   auto q = static_cast<const bf16*>(Q);
   auto k = static_cast<const bf16*>(K);
   cudaStream_t st = as_stream(stream);
@@ -239,13 +249,14 @@ const char* xattn_status_string(int status) {
   return "unknown status";
 }
 
-int xattn_version(void) { return 100; }
+int xattn_version(void) { return 200; }
 
-size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block) {
+size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block, int causal) {
   if (B < 0 || Hq < 0 || M < 0 || block != 128 || !stride_supported(stride) || M % block)
     return 0;
-  const size_t rp = (size_t)M / stride, nb = (size_t)M / block;
-  return (size_t)B * Hq * rp * (nb + 1) * sizeof(float);
+  const size_t rp = (size_t)M / stride;
+  return (score_part_entries(B, Hq, M, stride, block, causal) + (size_t)B * Hq * rp) *
+         sizeof(float);
 }
 
 int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C, int stride,
@@ -389,8 +400,9 @@ int xattn_select_group(const float* scores, const float* param, int rule, int B,
   return launch_status();
 }
 
-size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block) {
-  const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block);
+size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block,
+                                         int causal) {
+  const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block, causal);
   if (a == 0 && !(B == 0 || Hq == 0 || M == 0)) return 0;
   const size_t a_al = (a + 255) & ~(size_t)255;
   return a_al + xattn_select_workspace_size(B, Hq, block > 0 ? M / block : 0);
@@ -411,7 +423,7 @@ int xattn_score_select(const void* Q, const void* K, int B, int Hq, int Hkv, int
   if (worst >= (1LL << 31) || rows >= (1LL << 31) - 1) return XATTN_EUNSUPPORTED;
   if (!row_ptr || !nnz) return XATTN_EINVAL;
   if (rows > 0 && (!param || !col_idx)) return XATTN_EINVAL;
-  if (workspace_bytes < xattn_score_select_workspace_size(B, Hq, M, stride, block))
+  if (workspace_bytes < xattn_score_select_workspace_size(B, Hq, M, stride, block, causal))
     return XATTN_EINVAL;
   cudaStream_t st = as_stream(stream);
   if (rows == 0) {
@@ -420,7 +432,7 @@ int xattn_score_select(const void* Q, const void* K, int B, int Hq, int Hkv, int
     return XATTN_OK;
   }
   if (!workspace || ((uintptr_t)workspace & 15u) != 0) return XATTN_EINVAL;
-  const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block);
+  const size_t a = xattn_score_workspace_size(B, Hq, M, stride, block, causal);
   const size_t a_al = (a + 255) & ~(size_t)255;
   SelCut* cuts = reinterpret_cast<SelCut*>(static_cast<uint8_t*>(workspace) + a_al);
   FusedSelect fs;

@@ -41,7 +41,7 @@
  *     that ran out) set a per-device error word read by xattn_get_device_error.
  *   - An empty problem (B, H or M equal to 0) returns XATTN_OK and launches
  *     nothing.
- *   - Supported: block = 128; stride in {1, 2, 4, 8, 16}; C in {64, 128};
+ *   - Supported: block = 128; stride in {1, 2, 4, 8, 16, 32, 64}; C in {64, 128};
  *     M a multiple of 128; Hq a multiple of Hkv.
  */
 #ifndef XATTN_H
@@ -72,15 +72,21 @@ typedef enum {
 /* Static English description of a status code (never NULL). */
 XATTN_API const char* xattn_status_string(int status);
 
-/* Library ABI version (major*100 + minor). */
+/* Library ABI version (major*100 + minor); 200 since the workspace-size
+ * functions take the causal flag. */
 XATTN_API int xattn_version(void);
 
 /*
- * Workspace bytes xattn_score needs: fp32 per-(reshaped row, key block) partial
- * log-mass plus one fp32 log-sum-exp per reshaped row, i.e.
- * B*Hq*(M/stride)*(M/block+1)*4 bytes. Returns 0 for unsupported arguments.
+ * Workspace bytes xattn_score needs for the given `causal` flag: one fp32
+ * partial log-mass per (reshaped row, key block the row can see) plus one fp32
+ * log-sum-exp per reshaped row. With rp = M/stride and nb = M/block:
+ *   non-causal  B*Hq*rp*(nb + 1)*4 bytes
+ *   causal      B*Hq*(rp*(nb + 1)/2 + rp)*4 bytes  (about half: c <= r only)
+ * The workspace must be sized with the same `causal` value the scoring call
+ * gets. Returns 0 for unsupported arguments.
  */
-XATTN_API size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block);
+XATTN_API size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, int block,
+                                            int causal);
 
 /*
  * xattn_score - strided antidiagonal block scores [DuSA-Q2, XA-abs, XA-app].
@@ -100,8 +106,8 @@ XATTN_API size_t xattn_score_workspace_size(int B, int Hq, int M, int stride, in
  *   K           bf16 [B, Hkv, M, C]
  *   score_scale the scale of X; the usual value is 1/sqrt(stride*C)
  *   scores      fp32 [B, Hq, M/block, M/block] (output)
- *   workspace   device buffer of at least xattn_score_workspace_size() bytes,
- *               16-byte aligned; contents on entry are ignored
+ *   workspace   device buffer of at least xattn_score_workspace_size(..., causal)
+ *               bytes, 16-byte aligned; contents on entry are ignored
  */
 XATTN_API int xattn_score(const void* Q, const void* K, int B, int Hq, int Hkv, int M, int C,
                 int stride, int block, int causal, float score_scale,
@@ -187,10 +193,11 @@ XATTN_API int xattn_select_ex(const float* scores, const float* param, int rule,
                               size_t workspace_bytes, void* stream);
 
 /*
- * Workspace bytes xattn_score_select needs: the scoring workspace (rounded up
- * to 256 bytes) followed by the selection workspace.
+ * Workspace bytes xattn_score_select needs: the scoring workspace for the same
+ * `causal` flag (rounded up to 256 bytes) followed by the selection workspace.
  */
-XATTN_API size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block);
+XATTN_API size_t xattn_score_select_workspace_size(int B, int Hq, int M, int stride, int block,
+                                                   int causal);
 
 /*
  * xattn_score_select - xattn_score followed by xattn_select_ex, fused

@@ -118,6 +118,10 @@ def block_scores(q, k, stride: int, block: int, sigma: float, causal: bool,
     pair are summed and divided by g = block/stride, so that each block row sums
     to 1. Returns an [nb, nb] fp64 array (rows not in `rows` are left NaN;
     causal entries c > r are 0).
+
+    The logits of up to `chunk_blocks` consecutive query blocks are formed by one
+    matrix product (the same entries as one product per block, fewer passes over
+    the key view); every reshaped row is still softmax-normalised on its own.
     """
     M, C = q.shape
     if block % stride:
@@ -126,21 +130,29 @@ def block_scores(q, k, stride: int, block: int, sigma: float, causal: bool,
     qv, kv = strided_views(q, k, stride, antidiagonal)
     out = np.full((nb, nb), np.nan)
     rows = list(range(nb)) if rows is None else sorted(set(int(r) for r in rows))
-    for i in range(0, len(rows), chunk_blocks):
-        chunk = rows[i:i + chunk_blocks]
-        for r in chunk:
-            ri = slice(r * g, (r + 1) * g)
-            ncol = (r + 1) * g if causal else nb * g
-            X = sigma * (qv[ri] @ kv[:ncol].T)                 # [g, ncol]
-            if causal:
-                ii = np.arange(r * g, (r + 1) * g)[:, None]
-                jj = np.arange(ncol)[None, :]
-                X = np.where(jj <= ii, X, -np.inf)
-            X = X - X.max(axis=1, keepdims=True)               # row softmax (fp64)
-            P = np.exp(X)
-            P /= P.sum(axis=1, keepdims=True)
-            ncb = ncol // g
-            mass = P.reshape(g, ncb, g).sum(axis=(0, 2)) / g     # sum g x g, / g
+    # runs of consecutive query blocks, at most chunk_blocks long
+    runs, cur = [], []
+    for r in rows:
+        if cur and (r != cur[-1] + 1 or len(cur) == chunk_blocks):
+            runs.append(cur)
+            cur = []
+        cur.append(r)
+    if cur:
+        runs.append(cur)
+    for run in runs:
+        r0, r1 = run[0], run[-1]
+        ii = np.arange(r0 * g, (r1 + 1) * g)                   # reshaped query rows
+        ncol = (r1 + 1) * g if causal else nb * g
+        X = sigma * (qv[ii] @ kv[:ncol].T)                     # [rows, ncol]
+        if causal:
+            X = np.where(np.arange(ncol)[None, :] <= ii[:, None], X, -np.inf)
+        X = X - X.max(axis=1, keepdims=True)                   # row softmax (fp64)
+        P = np.exp(X)
+        P /= P.sum(axis=1, keepdims=True)
+        for r in run:
+            Pr = P[(r - r0) * g:(r - r0 + 1) * g]              # the g rows of block r
+            ncb = r + 1 if causal else nb                      # visible key blocks
+            mass = Pr[:, :ncb * g].reshape(g, ncb, g).sum(axis=(0, 2)) / g   # sum g x g, / g
             out[r, :] = 0.0
             out[r, :ncb] = mass
     return out

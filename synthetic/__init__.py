@@ -31,7 +31,9 @@ without drawing the others, and the bits never depend on which side asks.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from typing import Optional
 
 import numpy as np
@@ -200,23 +202,43 @@ def head_inputs(w: Workload, h: int, b: int = 0, seed: int = DEFAULT_SEED):
     return q_head_inputs(w, h, b, seed), k, v
 
 
-def layer_inputs(w: Workload, seed: int = DEFAULT_SEED, out=None):
+def layer_inputs(w: Workload, seed: int = DEFAULT_SEED, out=None, heads=None, threads=None):
     """Full (Q, K, V) bf16 bits: Q [B,Hq,M,C], K/V [B,Hkv,M,C] (uint16).
 
     `out` may hold three preallocated uint16 arrays (e.g. pinned host memory
-    viewed through numpy) to fill in place.
+    viewed through numpy) to fill in place. `heads` = (kv_lo, kv_hi) generates only
+    the KV heads kv_lo..kv_hi-1 and their query heads (the arrays then hold those
+    heads only, in order); every head is drawn from its own keyed stream, so a
+    slice has the same bits as the same heads of the whole layer. Heads are drawn
+    on `threads` host threads (default: the cores this process may use); the bits
+    do not depend on it.
     """
+    kv_lo, kv_hi = (0, w.Hkv) if heads is None else heads
+    g = w.group
+    nkv, nq = kv_hi - kv_lo, (kv_hi - kv_lo) * g
     if out is None:
-        Q = np.empty((w.B, w.Hq, w.M, w.C), np.uint16)
-        K = np.empty((w.B, w.Hkv, w.M, w.C), np.uint16)
-        V = np.empty((w.B, w.Hkv, w.M, w.C), np.uint16)
+        Q = np.empty((w.B, nq, w.M, w.C), np.uint16)
+        K = np.empty((w.B, nkv, w.M, w.C), np.uint16)
+        V = np.empty((w.B, nkv, w.M, w.C), np.uint16)
     else:
         Q, K, V = out
-    for b in range(w.B):
-        for kv in range(w.Hkv):
-            K[b, kv], V[b, kv] = kv_head_inputs(w, kv, b, seed)
-        for h in range(w.Hq):
-            Q[b, h] = q_head_inputs(w, h, b, seed)
+
+    def kv_job(b, kv):
+        K[b, kv - kv_lo], V[b, kv - kv_lo] = kv_head_inputs(w, kv, b, seed)
+
+    def q_job(b, h):
+        Q[b, h - kv_lo * g] = q_head_inputs(w, h, b, seed)
+
+    jobs = [(kv_job, b, kv) for b in range(w.B) for kv in range(kv_lo, kv_hi)] + \
+        [(q_job, b, h) for b in range(w.B) for h in range(kv_lo * g, kv_hi * g)]
+    n = threads or max(1, min(16, len(os.sched_getaffinity(0))))
+    if n == 1:
+        for f, b, i in jobs:
+            f(b, i)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(n) as ex:
+            for fut in [ex.submit(f, b, i) for f, b, i in jobs]:
+                fut.result()
     return Q, K, V
 
 

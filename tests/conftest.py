@@ -15,3 +15,11 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def repo_root():
     return ROOT
+
+
+def pytest_terminal_summary(terminalreporter):
+    from tests import parity
+    if parity.REPORT:
+        terminalreporter.section("mask parity report")
+        for line in parity.REPORT:
+            terminalreporter.write_line(line)

@@ -49,3 +49,33 @@ def dict_to_csr(kept_by_bh, B, Hq, nb):
     row_ptr[1:] = np.cumsum(counts)
     col = np.concatenate(lists).astype(np.int32)
     return (torch.from_numpy(row_ptr.astype(np.int32)).cuda(), torch.from_numpy(col).cuda())
+
+
+def poison_(t: torch.Tensor) -> torch.Tensor:
+    """Fill an output buffer with values no kernel writes (NaN for floating point,
+    -7 for int32, 0xFF bytes for raw workspaces), so that an element a kernel never
+    writes cannot pass for a result left behind by an earlier call."""
+    if t.dtype.is_floating_point:
+        t.fill_(float("nan"))
+    elif t.dtype == torch.uint8:
+        t.fill_(0xFF)
+    else:
+        t.fill_(-7)
+    return t
+
+
+def poisoned(shape, dtype=torch.float32, device="cuda") -> torch.Tensor:
+    return poison_(torch.empty(shape, dtype=dtype, device=device))
+
+
+def poisoned_like(t: torch.Tensor) -> torch.Tensor:
+    return poison_(torch.empty_like(t))
+
+
+def poison_buffers(bufs):
+    """poison_ every tensor of a Buffers set (outputs and workspaces)."""
+    for name in ("scores", "score_ws", "select_ws", "row_ptr", "col_idx", "nnz", "O", "lse"):
+        t = getattr(bufs, name)
+        if t is not None:
+            poison_(t)
+    return bufs

@@ -94,3 +94,33 @@ def assert_outputs_close(gpu: np.ndarray, ref: np.ndarray, what: str = "O"):
     assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, \
         f"{what}: max-abs {mx:.3e} (<= {OUT_MAX_ABS}), mean-abs {mean:.3e} (<= {OUT_MEAN_ABS})"
     return mx, mean
+
+
+def oracle_head_scores(args):
+    """The oracle's complete [nb, nb] block scores of one head, from bf16 bits
+    (a top-level function, so that a spawned worker process can run it)."""
+    qb, kb, stride, block, causal = args
+    q, k = orc.bf16_to_f64(qb), orc.bf16_to_f64(kb)
+    return orc.block_scores(q, k, stride, block, orc.default_score_scale(stride, q.shape[1]),
+                            causal)
+
+
+# Lines printed at the end of the pytest run (tests/conftest.py): every mask
+# exception of the full-size runs, and one summary line per configuration.
+REPORT: list = []
+
+
+def log_exception(config: str, head: int, exc) -> None:
+    """One mask exception from compare_row_mask: ("margin", r, c, margin) or
+    ("tie", r, c_oracle, c_gpu, score difference)."""
+    kind, r = exc[0], exc[1]
+    if kind == "margin":
+        REPORT.append(f"mask exception [{config}] head={head} row={r} block={exc[2]} "
+                      f"margin={exc[3]:+.3e} kind=margin")
+    else:
+        REPORT.append(f"mask exception [{config}] head={head} row={r} block={exc[2]}/{exc[3]} "
+                      f"score_diff={exc[4]:+.3e} kind=tie")
+
+
+def report(line: str) -> None:
+    REPORT.append(line)

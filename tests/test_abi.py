@@ -55,11 +55,17 @@ def test_status_strings_and_version():
 
 
 def test_workspace_sizes():
-    # partials (M/S x nb) + one LSE per reshaped row, fp32
-    assert xa.xattn_score_workspace_size(1, 32, 131072, 8) == 32 * 16384 * (1024 + 1) * 4
-    assert xa.xattn_score_workspace_size(1, 1, 2048, 4) == 512 * 17 * 4
-    assert xa.xattn_score_workspace_size(1, 1, 2048, 3) == 0
-    assert xa.xattn_score_workspace_size(1, 1, 2000, 8) == 0
+    # non-causal: partials (M/S x nb) + one LSE per reshaped row, fp32
+    assert xa.xattn_score_workspace_size(1, 32, 131072, 8, False) == 32 * 16384 * (1024 + 1) * 4
+    assert xa.xattn_score_workspace_size(1, 1, 2048, 4, False) == 512 * 17 * 4
+    # causal: the g rows of query block r keep r + 1 partials: g * nb(nb+1)/2 per head
+    assert xa.xattn_score_workspace_size(1, 32, 131072, 8, True) == \
+        32 * (16 * 1024 * 1025 // 2 + 16384) * 4
+    assert xa.xattn_score_workspace_size(2, 1, 2048, 4, True) == 2 * (32 * 16 * 17 // 2 + 512) * 4
+    assert xa.xattn_score_workspace_size(1, 1, 2048, 64, True) == (2 * 16 * 17 // 2 + 32) * 4
+    assert xa.xattn_score_workspace_size(1, 1, 2048, 3, True) == 0
+    assert xa.xattn_score_workspace_size(1, 1, 2000, 8, False) == 0
+    assert xa.xattn_score_workspace_size(1, 1, 2048, 128, True) == 0
     assert xa.xattn_select_workspace_size(1, 32, 1024) == 32 * 1024 * 12
     assert xa.xattn_select_workspace_size(1, 1, 1) == 256
     assert xa.max_kept(1, 2, 4, True) == 20 and xa.max_kept(1, 2, 4, False) == 32
@@ -81,7 +87,7 @@ def _score(**kw):
     (dict(C=96), xa.XATTN_EUNSUPPORTED),
     (dict(block=64, M=1024), xa.XATTN_EUNSUPPORTED),
     (dict(stride=3), xa.XATTN_EINVAL),
-    (dict(stride=32), xa.XATTN_EUNSUPPORTED),
+    (dict(stride=128), xa.XATTN_EUNSUPPORTED),
     (dict(stride=0), xa.XATTN_EINVAL),
     (dict(Q=None), xa.XATTN_EINVAL),
     (dict(ws=None), xa.XATTN_EINVAL),
@@ -184,8 +190,8 @@ def test_selftest_rejects_bad_limits():
 
 
 def test_fused_score_select_rejects_on_host():
-    assert xa.xattn_score_select_workspace_size(1, 2, 1024, 8) == \
-        ((xa.xattn_score_workspace_size(1, 2, 1024, 8) + 255) // 256 * 256 +
+    assert xa.xattn_score_select_workspace_size(1, 2, 1024, 8, True) == \
+        ((xa.xattn_score_workspace_size(1, 2, 1024, 8, True) + 255) // 256 * 256 +
          xa.xattn_select_workspace_size(1, 2, 8))
     args = [FAKE, FAKE, 1, 4, 2, 1024, 128, 8, 128, 1, 0.03, FAKE, 0, FAKE, FAKE, FAKE, 1 << 20,
             FAKE, FAKE, 1 << 40, None]

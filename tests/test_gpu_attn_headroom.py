@@ -19,7 +19,7 @@ import torch
 import oracle as orc
 import synthetic as sy
 from tests import parity as P
-from tests.gpu_util import bf16_to_np, to_dev
+from tests.gpu_util import poison_buffers, poisoned, poisoned_like, bf16_to_np, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -74,8 +74,8 @@ def test_dense_attention_far_from_first_block(C, causal, boost, heavy):
     M, Hq = 1024, 2
     Qb, Kb, Vb = _inputs(M, C, Hq, boost, heavy, seed=17)
     Q, K, V = to_dev(Qb), to_dev(Kb), to_dev(Vb)
-    O = torch.empty_like(Q)
-    lse = torch.empty((1, Hq, M), device="cuda")
+    O = poisoned_like(Q)
+    lse = poisoned((1, Hq, M))
     scale = 1 / math.sqrt(C)
     xa.xattn_dense_attn(Q, K, V, causal, scale, O, lse)
     got, gl = bf16_to_np(O), lse.cpu().numpy()
@@ -106,8 +106,8 @@ def test_sparse_attention_far_from_first_block(C, causal, boost, heavy):
             ptr.append(len(rows))
     rp = torch.tensor(ptr, dtype=torch.int32, device="cuda")
     ci = torch.tensor(rows, dtype=torch.int32, device="cuda")
-    O = torch.empty_like(Q)
-    lse = torch.empty((1, Hq, M), device="cuda")
+    O = poisoned_like(Q)
+    lse = poisoned((1, Hq, M))
     scale = 1 / math.sqrt(C)
     xa.xattn_sparse_attn(Q, K, V, rp, ci, causal, scale, O, lse)
     got, gl = bf16_to_np(O), lse.cpu().numpy()

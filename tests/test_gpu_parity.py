@@ -14,12 +14,16 @@ import torch
 import oracle as orc
 import synthetic as sy
 from tests import parity as P
-from tests.gpu_util import (bf16_to_np, csr_to_dict, device_inputs, dict_to_csr,
+from tests.gpu_util import (poison_buffers, poisoned, poisoned_like, bf16_to_np, csr_to_dict, device_inputs, dict_to_csr,
                             small_workload, to_dev)
 
 pytestmark = pytest.mark.gpu
 
 xa = pytest.importorskip("block_sparse_long_04_b200")
+
+
+def _alloc_poisoned(*a, **kw):
+    return poison_buffers(xa.Buffers.allocate(*a, **kw))
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -48,6 +52,10 @@ SCORE_CASES = [
     (256, 64, 1, 1, 16, False),
     (4096, 128, 8, 2, 8, True),     # several tiles in both directions
     (3200, 128, 4, 4, 4, True),     # M/S = 800: 7 tiles, ragged
+    (8320, 128, 2, 2, 32, False),   # M/S = 260: 3 tiles, ragged; 4 columns per block
+    (4096, 64, 2, 1, 32, True),
+    (16512, 128, 2, 1, 64, True),   # M/S = 258: 3 tiles, ragged; 2 columns per block
+    (2048, 64, 1, 1, 64, False),    # M/S = 32: one partial tile
 ]
 
 
@@ -57,7 +65,7 @@ def test_scores_match_oracle(M, C, Hq, Hkv, S, causal):
     (Qb, Kb, _), (Q, K, _) = device_inputs(w)
     nb = M // 128
     scores = torch.full((1, Hq, nb, nb), float("nan"), device="cuda")
-    ws = torch.empty(xa.xattn_score_workspace_size(1, Hq, M, S), dtype=torch.uint8, device="cuda")
+    ws = poisoned(xa.xattn_score_workspace_size(1, Hq, M, S, causal), torch.uint8)
     xa.xattn_score(Q, K, S, causal, orc.default_score_scale(S, C), scores, ws)
     got = scores.cpu().numpy()
     ref = _oracle_scores(Qb, Kb, w)
@@ -70,8 +78,8 @@ def test_score_scale_is_honoured():
     w = small_workload(1024, 128, 2, 1, 8, True)
     (Qb, Kb, _), (Q, K, _) = device_inputs(w)
     nb = 8
-    scores = torch.empty((1, 2, nb, nb), device="cuda")
-    ws = torch.empty(xa.xattn_score_workspace_size(1, 2, 1024, 8), dtype=torch.uint8, device="cuda")
+    scores = poisoned((1, 2, nb, nb))
+    ws = poisoned(xa.xattn_score_workspace_size(1, 2, 1024, 8, True), torch.uint8)
     for sc in (1.0 / 128, 1.0 / math.sqrt(128)):
         xa.xattn_score(Q, K, 8, True, sc, scores, ws)
         ref = _oracle_scores(Qb, Kb, w, scale=sc)
@@ -87,7 +95,7 @@ def _run_select(scores_np, tau, causal, cap=None):
     row_ptr = torch.full((B * Hq * nb + 1,), -7, dtype=torch.int32, device="cuda")
     col = torch.full((max(1, cap),), -7, dtype=torch.int32, device="cuda")
     nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8, device="cuda")
+    ws = poisoned(xa.xattn_select_workspace_size(B, Hq, nb), torch.uint8)
     xa.xattn_select(sc, t, causal, row_ptr, col, nnz, ws)
     return row_ptr.cpu().numpy(), col.cpu().numpy(), int(nnz.item())
 
@@ -98,6 +106,8 @@ def _check_masks(row_ptr, col, scores_ref, tau, causal, Hq, nb, log):
         for r in range(nb):
             gcols = col[row_ptr[h * nb + r]:row_ptr[h * nb + r + 1]]
             exc, f = P.compare_row_mask(gcols, scores_ref[h][r], r, float(tau[h]), causal)
+            for x in exc:
+                P.log_exception(f"selection nb={nb} causal={causal}", h, x)
             log += exc
             fails += f
     return fails
@@ -168,8 +178,8 @@ def test_sparse_attention_on_oracle_mask(M, C, Hq, Hkv, causal):
     sc = _oracle_scores(Qb, Kb, w)
     kept = orc.layer_select(sc, np.full(Hq, 0.7), causal)
     row_ptr, col = dict_to_csr(kept, 1, Hq, nb)
-    O = torch.empty_like(Q)
-    lse = torch.empty((1, Hq, M), device="cuda")
+    O = poisoned_like(Q)
+    lse = poisoned((1, Hq, M))
     xa.xattn_sparse_attn(Q, K, V, row_ptr, col, causal, 1 / math.sqrt(C), O, lse)
     ref = orc.layer_sparse_attention(Qb, Kb, Vb, Hkv, kept, 128, causal, 1 / math.sqrt(C))
     got, glse = bf16_to_np(O), lse.cpu().numpy()
@@ -182,8 +192,8 @@ def test_sparse_attention_on_oracle_mask(M, C, Hq, Hkv, causal):
 def test_dense_attention_matches_oracle(M, C, Hq, Hkv, causal):
     w = small_workload(M, C, Hq, Hkv, 8, causal)
     (Qb, Kb, Vb), (Q, K, V) = device_inputs(w)
-    O = torch.empty_like(Q)
-    lse = torch.empty((1, Hq, M), device="cuda")
+    O = poisoned_like(Q)
+    lse = poisoned((1, Hq, M))
     xa.xattn_dense_attn(Q, K, V, causal, 1 / math.sqrt(C), O, lse)
     got = bf16_to_np(O)
     grp = Hq // Hkv
@@ -204,8 +214,8 @@ def test_attention_skips_invalid_entries_and_empty_rows():
     rp = torch.tensor(np.concatenate([[0], np.cumsum([len(x) for x in lists])]), dtype=torch.int32,
                       device="cuda")
     ci = torch.tensor(sum(lists, []), dtype=torch.int32, device="cuda")
-    O = torch.empty_like(Q)
-    lse = torch.empty((1, Hq, M), device="cuda")
+    O = poisoned_like(Q)
+    lse = poisoned((1, Hq, M))
     xa.xattn_sparse_attn(Q, K, V, rp, ci, True, 0.125, O, lse)
     got, gl = bf16_to_np(O)[0, 0], lse.cpu().numpy()[0, 0]
     assert (got[:128] == 0).all() and np.isneginf(gl[:128]).all()
@@ -245,7 +255,7 @@ def test_sparse_attention_list_order_does_not_matter(causal):
             ptr.append(len(rows))
     rp = torch.tensor(ptr, dtype=torch.int32, device="cuda")
     ci = torch.tensor(rows, dtype=torch.int32, device="cuda")
-    O = torch.empty_like(Q)
+    O = poisoned_like(Q)
     xa.xattn_sparse_attn(Q, K, V, rp, ci, causal, 1 / math.sqrt(C), O)
     got = bf16_to_np(O)
     grp = Hq // Hkv
@@ -256,7 +266,7 @@ def test_sparse_attention_list_order_does_not_matter(causal):
 
 
 def _pipeline(w, Q, K, V, tau, with_lse=False):
-    bufs = xa.Buffers.allocate(w.B, w.Hq, w.M, w.C, w.stride, w.causal, with_lse=with_lse)
+    bufs = _alloc_poisoned(w.B, w.Hq, w.M, w.C, w.stride, w.causal, with_lse=with_lse)
     t = torch.from_numpy(np.asarray(tau, np.float32)).cuda()
     xa.xattn_prefill(Q, K, V, t, w.stride, w.causal, bufs)
     torch.cuda.synchronize()
@@ -285,6 +295,8 @@ def test_pipeline_end_to_end_small(name, kw):
         for r in range(nb):
             gcols = col[row_ptr[h * nb + r]:row_ptr[h * nb + r + 1]]
             e, f = P.compare_row_mask(gcols, ref_s[(0, h)][r], r, float(tau[h]), w.causal)
+            for x in e:
+                P.log_exception(f"pipeline {name} M={w.M} S={w.stride}", h, x)
             log += e
             fails += f
     assert not fails, fails[:5]
@@ -298,7 +310,7 @@ def test_pipeline_end_to_end_small(name, kw):
     for h in range(w.Hq):
         P.assert_outputs_close(got_o[0, h], ref_gk[(0, h)][0], f"O (gpu mask) head {h}")
     rp2, col2 = dict_to_csr(ok, 1, w.Hq, nb)
-    O2 = torch.empty_like(Q)
+    O2 = poisoned_like(Q)
     xa.xattn_sparse_attn(Q, K, V, rp2, col2, w.causal, scale, O2)
     ref_ok = orc.layer_sparse_attention(Qb, Kb, Vb, w.Hkv, ok, 128, w.causal, scale)
     got2 = bf16_to_np(O2)
@@ -310,7 +322,7 @@ def test_tau_one_equals_dense():
     w = small_workload(1024, 128, 2, 1, 8, True)
     (_, _, _), (Q, K, V) = device_inputs(w)
     bufs = _pipeline(w, Q, K, V, [1.0, 1.0])
-    O = torch.empty_like(Q)
+    O = poisoned_like(Q)
     xa.xattn_dense_attn(Q, K, V, True, 1 / math.sqrt(128), O)
     assert torch.equal(O, bufs.O)
     assert int(bufs.nnz.item()) == 2 * 8 * 9 // 2
@@ -327,11 +339,11 @@ def test_repeatable_bits():
 
 
 def test_empty_problem_is_a_no_op():
-    Q = torch.empty((1, 2, 0, 128), dtype=torch.bfloat16, device="cuda")
-    O = torch.empty_like(Q)
+    Q = poisoned((1, 2, 0, 128), torch.bfloat16)
+    O = poisoned_like(Q)
     xa.xattn_dense_attn(Q, Q[:, :1], Q[:, :1], True, 0.1, O)
-    scores = torch.empty((1, 2, 0, 0), device="cuda")
-    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    scores = poisoned((1, 2, 0, 0))
+    ws = poisoned(16, torch.uint8)
     xa.xattn_score(Q, Q[:, :1], 8, True, 0.1, scores, ws)
     assert xa.xattn_get_device_error() == xa.XATTN_OK
 

@@ -10,7 +10,7 @@ import torch
 
 import oracle as orc
 from tests import parity as P
-from tests.gpu_util import bf16_to_np, csr_to_dict, device_inputs, dict_to_csr, small_workload
+from tests.gpu_util import poison_buffers, poisoned, poisoned_like, bf16_to_np, csr_to_dict, device_inputs, dict_to_csr, small_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -30,23 +30,24 @@ def _cuda():
     (1152, 128, 4, 2, 8, True),
     (1024, 128, 2, 1, 4, False),
     (640, 64, 2, 2, 16, True),
+    (8320, 128, 2, 1, 64, True),
 ])
 def test_diagonal_pattern_scores(M, C, Hq, Hkv, S, causal):
     w = small_workload(M, C, Hq, Hkv, S, causal)
     (Qb, Kb, _), (Q, K, _) = device_inputs(w)
     nb = M // 128
     sig = orc.default_score_scale(S, C)
-    scores = torch.empty((1, Hq, nb, nb), device="cuda")
-    ws = torch.empty(xa.xattn_score_workspace_size(1, Hq, M, S), dtype=torch.uint8, device="cuda")
+    scores = poisoned((1, Hq, nb, nb))
+    ws = poisoned(xa.xattn_score_workspace_size(1, Hq, M, S, causal), torch.uint8)
     xa.xattn_score_ex(Q, K, S, causal, xa.XATTN_PATTERN_DIAGONAL, sig, scores, ws)
     diag = scores.cpu().numpy()
     ref = orc.layer_block_scores(Qb, Kb, Hkv, S, 128, sig, causal, antidiagonal=False)
     for h in range(Hq):
         P.assert_scores_close(diag[0, h], ref[(0, h)], f"diagonal scores head {h}")
     # and the antidiagonal pattern through the same entry point is xattn_score
-    anti = torch.empty_like(scores)
+    anti = poisoned_like(scores)
     xa.xattn_score_ex(Q, K, S, causal, xa.XATTN_PATTERN_ANTIDIAGONAL, sig, anti, ws)
-    base = torch.empty_like(scores)
+    base = poisoned_like(scores)
     xa.xattn_score(Q, K, S, causal, sig, base, ws)
     assert torch.equal(anti, base)
     if M >= 1024:
@@ -57,10 +58,10 @@ def _select_ex(scores_np, param, rule, causal):
     B, Hq, nb, _ = scores_np.shape
     sc = torch.from_numpy(np.ascontiguousarray(scores_np, dtype=np.float32)).cuda()
     pr = torch.tensor(param, dtype=torch.float32, device="cuda")
-    row_ptr = torch.empty(B * Hq * nb + 1, dtype=torch.int32, device="cuda")
-    col = torch.empty(xa.max_kept(B, Hq, nb, causal), dtype=torch.int32, device="cuda")
+    row_ptr = poisoned(B * Hq * nb + 1, torch.int32)
+    col = poisoned(xa.max_kept(B, Hq, nb, causal), torch.int32)
     nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8, device="cuda")
+    ws = poisoned(xa.xattn_select_workspace_size(B, Hq, nb), torch.uint8)
     xa.xattn_select_ex(sc, pr, rule, causal, row_ptr, col, nnz, ws)
     return row_ptr.cpu().numpy(), col.cpu().numpy(), int(nnz.item())
 
@@ -99,10 +100,10 @@ def test_threshold_rule_equals_select():
     a = _select_ex(s, [0.9, 0.6], xa.XATTN_SELECT_THRESHOLD, True)
     sc = torch.from_numpy(s).cuda()
     tau = torch.tensor([0.9, 0.6], device="cuda")
-    row_ptr = torch.empty(Hq * nb + 1, dtype=torch.int32, device="cuda")
-    col = torch.empty(xa.max_kept(1, Hq, nb, True), dtype=torch.int32, device="cuda")
+    row_ptr = poisoned(Hq * nb + 1, torch.int32)
+    col = poisoned(xa.max_kept(1, Hq, nb, True), torch.int32)
     nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(xa.xattn_select_workspace_size(1, Hq, nb), dtype=torch.uint8, device="cuda")
+    ws = poisoned(xa.xattn_select_workspace_size(1, Hq, nb), torch.uint8)
     xa.xattn_select(sc, tau, True, row_ptr, col, nnz, ws)
     n = int(nnz.item())
     assert a[2] == n
@@ -116,11 +117,12 @@ def test_threshold_rule_equals_select():
     (1024, 128, 2, 1, 4, False, 1),
     (4096, 128, 4, 2, 16, True, 1),
 ])
-def test_fused_score_select_equals_two_calls(M, C, Hq, Hkv, S, causal, B):
+def test_fused_score_select_equals_two_calls_and_oracle(M, C, Hq, Hkv, S, causal, B):
     w = small_workload(M, C, Hq, Hkv, S, causal).with_(B=B)
-    _, (Q, K, _) = device_inputs(w)
+    (Qb, Kb, _), (Q, K, _) = device_inputs(w)
     nb = M // 128
     sig = orc.default_score_scale(S, C)
+    ref_s = orc.layer_block_scores(Qb, Kb, Hkv, S, 128, sig, causal)
     rules = ((xa.XATTN_SELECT_THRESHOLD, [0.9, 0.7, 0.95, 0.6][:Hq]),
              (xa.XATTN_SELECT_TOPK, [3.0, 1.0, 5.0, 2.0][:Hq]),
              (xa.XATTN_SELECT_RATIO, [0.25, 0.5, 0.1, 1.0][:Hq]))
@@ -128,40 +130,61 @@ def test_fused_score_select_equals_two_calls(M, C, Hq, Hkv, S, causal, B):
     for rule, prm in rules:
         param = torch.tensor(prm, dtype=torch.float32, device="cuda")
         # reference: the two separate calls
-        sc1 = torch.empty((B, Hq, nb, nb), device="cuda")
-        ws1 = torch.empty(xa.xattn_score_workspace_size(B, Hq, M, S), dtype=torch.uint8,
-                          device="cuda")
+        sc1 = poisoned((B, Hq, nb, nb))
+        ws1 = poisoned(xa.xattn_score_workspace_size(B, Hq, M, S, causal), torch.uint8)
         xa.xattn_score(Q, K, S, causal, sig, sc1, ws1)
-        rp1 = torch.empty(B * Hq * nb + 1, dtype=torch.int32, device="cuda")
+        rp1 = poisoned(B * Hq * nb + 1, torch.int32)
         ci1 = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
         nz1 = torch.zeros(1, dtype=torch.int32, device="cuda")
-        wss = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8,
-                          device="cuda")
+        wss = poisoned(xa.xattn_select_workspace_size(B, Hq, nb), torch.uint8)
         xa.xattn_select_ex(sc1, param, rule, causal, rp1, ci1, nz1, wss)
         # fused
-        sc2 = torch.empty_like(sc1)
-        rp2 = torch.empty_like(rp1)
+        sc2 = poisoned_like(sc1)
+        rp2 = poisoned_like(rp1)
         ci2 = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
         nz2 = torch.zeros(1, dtype=torch.int32, device="cuda")
-        ws2 = torch.empty(xa.xattn_score_select_workspace_size(B, Hq, M, S), dtype=torch.uint8,
-                          device="cuda")
+        ws2 = poisoned(xa.xattn_score_select_workspace_size(B, Hq, M, S, causal), torch.uint8)
         xa.xattn_score_select(Q, K, param, rule, S, causal, sig, sc2, rp2, ci2, nz2, ws2)
         torch.cuda.synchronize()
         n = int(nz1.item())
         assert torch.equal(sc1, sc2)
         assert int(nz2.item()) == n and torch.equal(rp1, rp2)
         assert torch.equal(ci1[:n], ci2[:n])
+        # the fused lists against the oracle: the threshold rule on the oracle's own
+        # scores (mask-exception rules), Top-K / ratio (ranking only) exactly on the
+        # scores the GPU ranked
+        rp, ci = rp2.cpu().numpy(), ci2.cpu().numpy()
+        got_s = sc2.cpu().numpy().astype(np.float64)
+        fails = []
+        for b in range(B):
+            for h in range(Hq):
+                bh = b * Hq + h
+                for r in range(nb):
+                    gk = ci[rp[bh * nb + r]:rp[bh * nb + r + 1]]
+                    if rule == xa.XATTN_SELECT_THRESHOLD:
+                        e, f = P.compare_row_mask(gk, ref_s[(b, h)][r], r, float(np.float32(prm[h])),
+                                                  causal)
+                        for x in e:
+                            P.log_exception(f"fused M={M} S={S} B={B}", h, x)
+                        fails += f
+                    elif rule == xa.XATTN_SELECT_TOPK:
+                        want = orc.select_row_topk(got_s[b, h, r], r, int(prm[h]), causal)
+                        assert gk.tolist() == want.tolist(), (b, h, r)
+                    else:
+                        want = orc.select_row_ratio(got_s[b, h, r], r, float(np.float32(prm[h])),
+                                                    causal)
+                        assert gk.tolist() == want.tolist(), (b, h, r)
+        assert not fails, fails[:5]
 
 
 def _select_group(scores_np, param, rule, Hkv, causal):
     B, Hq, nb, _ = scores_np.shape
     sc = torch.from_numpy(np.ascontiguousarray(scores_np, dtype=np.float32)).cuda()
     pr = torch.tensor(param, dtype=torch.float32, device="cuda")
-    row_ptr = torch.empty(B * Hkv * nb + 1, dtype=torch.int32, device="cuda")
+    row_ptr = poisoned(B * Hkv * nb + 1, torch.int32)
     col = torch.full((xa.max_kept(B, Hkv, nb, causal),), -7, dtype=torch.int32, device="cuda")
     nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(xa.xattn_select_group_workspace_size(B, Hq, Hkv, nb), dtype=torch.uint8,
-                     device="cuda")
+    ws = poisoned(xa.xattn_select_group_workspace_size(B, Hq, Hkv, nb), torch.uint8)
     xa.xattn_select_group(sc, pr, rule, Hkv, causal, row_ptr, col, nnz, ws)
     return row_ptr.cpu().numpy(), col.cpu().numpy(), int(nnz.item())
 
@@ -218,8 +241,8 @@ def test_group_attention_matches_oracle(M, C, Hq, Hkv, causal):
     kept = orc.layer_select(sc, np.full(Hq, 0.7), causal)
     union = orc.layer_select_group(kept, Hq, Hkv)
     row_ptr, col = dict_to_csr(union, 1, Hkv, nb)
-    O = torch.empty_like(Q)
-    lse = torch.empty((1, Hq, M), device="cuda")
+    O = poisoned_like(Q)
+    lse = poisoned((1, Hq, M))
     xa.xattn_sparse_attn_group(Q, K, V, row_ptr, col, causal, 1 / math.sqrt(C), O, lse)
     grp = Hq // Hkv
     by_head = {(0, h): union[(0, h // grp)] for h in range(Hq)}
@@ -238,11 +261,10 @@ def test_group_selection_capacity_error_is_reported():
     s /= s.sum(-1, keepdims=True)
     sc = torch.from_numpy(s).cuda()
     pr = torch.ones(Hq, dtype=torch.float32, device="cuda")
-    row_ptr = torch.empty(B * Hkv * nb + 1, dtype=torch.int32, device="cuda")
+    row_ptr = poisoned(B * Hkv * nb + 1, torch.int32)
     col = torch.full((10,), -7, dtype=torch.int32, device="cuda")
     nnz = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = torch.empty(xa.xattn_select_group_workspace_size(B, Hq, Hkv, nb), dtype=torch.uint8,
-                     device="cuda")
+    ws = poisoned(xa.xattn_select_group_workspace_size(B, Hq, Hkv, nb), torch.uint8)
     xa.xattn_select_group(sc, pr, xa.XATTN_SELECT_THRESHOLD, Hkv, True, row_ptr, col, nnz, ws)
     torch.cuda.synchronize()
     assert int(nnz.item()) == B * Hkv * nb * (nb + 1) // 2

@@ -18,6 +18,8 @@ import numpy as np
 import pytest
 import torch
 
+from tests.gpu_util import poison_buffers, poisoned, poisoned_like
+
 from block_sparse_long_04_b200 import build as _build
 
 _build.build()
@@ -52,8 +54,7 @@ def test_noalloc_select_equals_select_on_consecutive_calls():
         scores = _scores(seed, Hq, nb, causal)
         tau = torch.tensor(taus, dtype=torch.float32, device="cuda")
         ref = _outputs(Hq, nb, causal)
-        ws = torch.empty(xa.xattn_select_workspace_size(1, Hq, nb), dtype=torch.uint8,
-                         device="cuda")
+        ws = poisoned(xa.xattn_select_workspace_size(1, Hq, nb), torch.uint8)
         xa.xattn_select(scores, tau, causal, *ref, ws)
         got = _outputs(Hq, nb, causal)
         rp, ci, nz = got
@@ -109,7 +110,7 @@ def test_noalloc_select_fills_its_whole_scratch():
     ref = (torch.full((B * Hq * nb + 1,), -1, dtype=torch.int32, device="cuda"),
            torch.full((cap,), -1, dtype=torch.int32, device="cuda"),
            torch.full((1,), -1, dtype=torch.int32, device="cuda"))
-    ws = torch.empty(xa.xattn_select_workspace_size(B, Hq, nb), dtype=torch.uint8, device="cuda")
+    ws = poisoned(xa.xattn_select_workspace_size(B, Hq, nb), torch.uint8)
     xa.xattn_select(s, tau, causal, *ref, ws)
     got = tuple(torch.full_like(t, -1) for t in ref)
     rc = _call([s.data_ptr(), tau.data_ptr(), got[0].data_ptr(), got[1].data_ptr(),
