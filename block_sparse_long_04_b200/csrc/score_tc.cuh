@@ -42,11 +42,17 @@ namespace xattn {
 
 constexpr int kScoreTcThreads = 384;
 
-template <int BN>
+// PAIR: 0 = one CTA per tile; 1 = a CTA pair (cta_group::2) over two query heads
+// of one KV group (same tile, same key columns); 2 = a CTA pair over two
+// neighbouring row tiles of one head. In a pair each CTA holds its own 128 query
+// rows and half of every BN-column key tile, so each SM reads and stores half the
+// key bytes of a single-CTA tile.
+template <int BN, int PAIR = 0>
 struct ScoreTc {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = PAIR ? 6 : (BN == 256 ? 4 : 6);
   static constexpr int kQBytes = 128 * 128;              // 128 rows x 64 bf16
-  static constexpr int kKBytes = BN * 128;               // BN rows x 64 bf16
+  static constexpr int kKRows = PAIR ? BN / 2 : BN;      // key rows this CTA loads
+  static constexpr int kKBytes = kKRows * 128;           // kKRows rows x 64 bf16
   static constexpr int kStageBytes = kQBytes + kKBytes;
   static constexpr int kOffBar = kStages * kStageBytes;
   static constexpr int kOffLse = kOffBar + 256;
@@ -55,15 +61,21 @@ struct ScoreTc {
   static constexpr int kTmemCols = 2 * BN;
 };
 
-template <int C, int G, int BN, bool SELECT>
+template <int C, int G, int BN, bool SELECT, int PAIR>
 __global__ void __launch_bounds__(kScoreTcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 int Hq, int Hkv, int M, int causal, int diagonal, float scale_log2,
                 float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores,
                 const float* __restrict__ sel_param, int sel_rule, SelCut* __restrict__ cuts);
 
-static_assert(ScoreTc<128>::kOffBar >= kSelMaxNb * 8 + 64 && ScoreTc<256>::kOffBar >= kSelMaxNb * 8 + 64,
-              "the stage ring must hold the fused selection's sort keys");
+// the fused selection's layout inside the idle stage ring: sort keys / ranks,
+// the fp64 scan scratch and its first-hit word, then the cut search state
+constexpr int kSelRingRed = kSelMaxNb * 8;
+constexpr int kSelRingRadix = kSelMaxNb * 8 + 256;
+static_assert(ScoreTc<128>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix) &&
+              ScoreTc<256>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix) &&
+              ScoreTc<256, 1>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix),
+              "the stage ring must hold the fused selection's keys and search state");
 
 // Offset of reshaped row ip's partial log-masses in the workspace. Non-causal:
 // nb entries per row. Causal: the g = G rows of query block r hold only the
@@ -76,13 +88,13 @@ __device__ __forceinline__ size_t part_row(int bh, int ip, int rp, int nb, int c
   return (size_t)bh * ((size_t)rp * (nb + 1) / 2) + G * (r * (r + 1) / 2) + i * (r + 1);
 }
 
-template <int C, int G, int BN, bool SELECT>
+template <int C, int G, int BN, bool SELECT, int PAIR>
 __global__ void __launch_bounds__(kScoreTcThreads, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 int Hq, int Hkv, int M, int causal, int diagonal, float scale_log2,
                 float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores,
                 const float* __restrict__ sel_param, int sel_rule, SelCut* __restrict__ cuts) {
-  using L = ScoreTc<BN>;
+  using L = ScoreTc<BN, PAIR>;
   constexpr int ST = L::kStages;
   constexpr int S = 128 / G;
   constexpr int NCH = S * C / 64;       // 64-wide chunks of the reshaped width
@@ -106,79 +118,137 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int rp = M / S;
   const int nb = M / 128;
   const int RT = (rp + 127) / 128;
-  const int t = causal ? (RT - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int bh = blockIdx.y;
+  // this CTA's rank in its pair (0 = the leader, which issues the pair's MMAs)
+  const int crank = PAIR ? (int)cluster_ctarank() : 0;
+  const bool leader = crank == 0;
+  int t, bh, t_cols;   // row tile, (batch, query head), the tile whose columns the pair sweeps
+  if (PAIR == 1) {
+    // heads 2j and 2j+1 share a KV head (Hq/Hkv even): same tile, same columns
+    const int tt = (int)blockIdx.x >> 1;
+    t = t_cols = causal ? RT - 1 - tt : tt;
+    bh = 2 * (int)blockIdx.y + crank;
+  } else if (PAIR == 2) {
+    // neighbouring row tiles of one head; the pair sweeps the longer one's columns,
+    // and a CTA past the last tile (RT odd) only lends its half of the key tiles
+    const int slot = (int)blockIdx.x;
+    t = causal ? RT - 1 - slot : slot;
+    t_cols = causal ? RT - 1 - (slot & ~1) : (slot | 1);
+    bh = blockIdx.y;
+  } else {
+    t = t_cols = causal ? (RT - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    bh = blockIdx.y;
+  }
+  const bool dummy = t < 0 || t >= RT;
   const int b = bh / Hq, h = bh % Hq, kvh = h / (Hq / Hkv);
-  const int i0 = t * 128;
-  // column tiles: causal needs columns up to i0 + 127
-  const int njt = causal ? min((i0 + 127) / BN + 1, (rp + BN - 1) / BN) : (rp + BN - 1) / BN;
+  const int i0 = dummy ? RT * 128 : t * 128;          // a dummy CTA's rows are all >= rp
+  const int iq = dummy ? min(max(t_cols, 0), RT - 1) * 128 : i0;   // rows its Q loads read
+  // column tiles: causal needs columns up to (row tile + 1) * 128 - 1
+  const int njt = causal ? min((t_cols * 128 + 127) / BN + 1, (rp + BN - 1) / BN)
+                         : (rp + BN - 1) / BN;
   const int total = njt * NCH;
 
   if (tid == 0) {
     for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], PAIR ? 16 : 8);   // the epilogue warps of the whole pair
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, L::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, L::kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (tid == 64) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync();   // both CTAs' barriers exist before either signals the other's
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const int yq = bh * rp + i0;
-      const int yk0 = (b * Hkv + kvh) * rp;
+      const int yq = bh * rp + iq;
+      const int yk0 = (b * Hkv + kvh) * rp + crank * L::kKRows;
+      // a pair's loads complete on the leader's `full` barriers
+      const uint32_t full_lead = PAIR ? mapa_shared(full, 0) : 0u;
       int it = 0;
       for (; it < total; ++it) {
         const int st = it % ST;
         if (it >= ST && !mbar_wait(&empty[st], ((it / ST) - 1) & 1, abort_flag)) break;
         const int jt = it / NCH, q = it % NCH;
         const int s = (q * 64) / C, d0 = (q * 64) % C;
-        mbar_expect_tx(&full[st], L::kStageBytes);
         const uint32_t dst = sbase + st * L::kStageBytes;
         // antidiagonal: query rows reversed inside the stride group; diagonal: forward
-        tma_load_2d(dst, &tmQ, (diagonal ? s : S - 1 - s) * C + d0, yq, &full[st]);
-        tma_load_2d(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, &full[st]);
+        const int xq = (diagonal ? s : S - 1 - s) * C + d0;
+        if (PAIR) {
+          if (leader) mbar_expect_tx(&full[st], 2 * L::kStageBytes);
+          tma_load_2d_pair(dst, &tmQ, xq, yq, full_lead + st * 8);
+          tma_load_2d_pair(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, full_lead + st * 8);
+        } else {
+          mbar_expect_tx(&full[st], L::kStageBytes);
+          tma_load_2d(dst, &tmQ, xq, yq, &full[st]);
+          tma_load_2d(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, &full[st]);
+        }
       }
-      volatile int no_abort = 0;
-      for (int jj = (it > ST ? it - ST : 0); jj < it; ++jj)
-        mbar_wait(&full[jj % ST], (jj / ST) & 1, &no_abort);
+      // drain: every load issued must land before the CTA may exit (the leader's
+      // barriers also count the other CTA's loads; that CTA leaves only after the
+      // cluster barrier at the end, which the leader reaches after this drain)
+      if (leader) {
+        volatile int no_abort = 0;
+        for (int jj = (it > ST ? it - ST : 0); jj < it; ++jj)
+          mbar_wait(&full[jj % ST], (jj / ST) & 1, &no_abort);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
-      bool ok = true;
-      for (int it = 0; ok && it < total; ++it) {
-        const int st = it % ST;
-        const int jt = it / NCH, q = it % NCH;
-        const int buf = jt & 1;
-        if (q == 0 && jt >= 2) {
-          if (!(ok = mbar_wait(&acc_empty[buf], ((jt / 2) - 1) & 1, abort_flag))) break;
-        }
-        if (!(ok = mbar_wait(&full[st], (it / ST) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t a0 = sbase + st * L::kStageBytes;
-        const uint32_t b0 = a0 + L::kQBytes;
+      // a pair: the leader issues M = 256 MMAs (each CTA's 128 rows against both
+      // halves of the key tile) and signals both CTAs' barriers; the other CTA's
+      // issuer only waits for the pair's last MMA
+      if (leader) {
+        constexpr uint32_t idesc = idesc_bf16_f32(PAIR ? 256 : 128, BN, false, false);
+        bool ok = true;
+        for (int it = 0; ok && it < total; ++it) {
+          const int st = it % ST;
+          const int jt = it / NCH, q = it % NCH;
+          const int buf = jt & 1;
+          if (q == 0 && jt >= 2) {
+            if (!(ok = mbar_wait(&acc_empty[buf], ((jt / 2) - 1) & 1, abort_flag))) break;
+          }
+          if (!(ok = mbar_wait(&full[st], (it / ST) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t a0 = sbase + st * L::kStageBytes;
+          const uint32_t b0 = a0 + L::kQBytes;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16_ss(tmem + buf * BN, smem_desc_sw128(a0 + kk * 32, 16, 1024),
-                     smem_desc_sw128(b0 + kk * 32, 16, 1024), idesc, (q > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&empty[st]);
-        if (q == NCH - 1) mma_commit(&acc_full[buf]);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t db = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            if (PAIR) mma_f16_ss_pair(tmem + buf * BN, da, db, idesc, (q > 0 || kk > 0) ? 1u : 0u);
+            else mma_f16_ss(tmem + buf * BN, da, db, idesc, (q > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (PAIR) {
+            mma_commit_pair(&empty[st]);
+            if (q == NCH - 1) mma_commit_pair(&acc_full[buf]);
+          } else {
+            mma_commit(&empty[st]);
+            if (q == NCH - 1) mma_commit(&acc_full[buf]);
+          }
+        }
+        if (PAIR) mma_commit_pair(drain);
+        else mma_commit(drain);
       }
-      mma_commit(drain);
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
@@ -207,7 +277,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (ch == 128 / CH - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          if (lane == 0) {
+            if (PAIR) mbar_arrive_cluster(mapa_shared(&acc_empty[buf], 0));   // the leader's
+            else mbar_arrive(&acc_empty[buf]);
+          }
         }
         const int j0 = jt * BN + hh * 128 + ch * CH;
 #pragma unroll
@@ -284,8 +357,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int et = tid - 128;
       if (done_ok) {
         uint64_t* keys = reinterpret_cast<uint64_t*>(smem);             // the idle stage ring
-        double* red = reinterpret_cast<double*>(smem + kSelMaxNb * 8);
+        double* red = reinterpret_cast<double*>(smem + kSelRingRed);
         int* first_hit = reinterpret_cast<int*>(red + 4);
+        SelRadix* st = reinterpret_cast<SelRadix*>(smem + kSelRingRadix);
         auto sync = [] { asm volatile("bar.sync 2, 128;" ::: "memory"); };
         for (int k = 0; k < 128 / G; ++k) {
           const int r = i0 / G + k;
@@ -293,7 +367,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int n = causal ? r + 1 : nb;
           const SelCut cut = select_row_cut<128>(scores + ((size_t)bh * nb + r) * nb, n, r,
                                                  sel_param[h], sel_rule, keys, red,
-                                                 first_hit, et, sync);
+                                                 first_hit, st, et, sync);
           if (et == 0) cuts[(size_t)bh * nb + r] = cut;
         }
       } else {
@@ -304,11 +378,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   }
 
-  __syncthreads();
+  tc_fence_before();
+  if (PAIR) cluster_sync();   // neither CTA leaves while the other may still touch its memory
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem, L::kTmemCols);
+    else tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 

@@ -3,10 +3,10 @@
 // is the prefix of the descending order).
 //
 // Three launches:
-//   select_count  one CTA per row (b, h, r): sort the row's candidate scores
-//                 (descending, ties to the smaller block index) with a bitonic
-//                 network in shared memory, prefix-sum them in fp64, find the
-//                 cut (the first position whose cumulative sum reaches tau), and
+//   select_count  one CTA per row (b, h, r): find the cut of the row's candidate
+//                 scores (descending, ties to the smaller block index): the first
+//                 position whose cumulative sum reaches tau, by a radix search
+//                 over the score ranks with exact per-bin masses (no sort), and
 //                 record the cut key (score, index) and the kept count (with the
 //                 diagonal added if it falls below the cut).
 //   select_scan   one CTA: exclusive scan of the counts into row_ptr and nnz;
@@ -91,9 +91,12 @@ __device__ __forceinline__ double group_exclusive_scan_f64(double v, double* red
     const double y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
+  // the exclusive value is the previous lane's inclusive one (not x - v, which
+  // is NaN when v is infinite)
+  double before = __shfl_up_sync(0xffffffffu, x, 1);
+  if (lane == 0) before = 0.0;
   if (lane == 31) red[warp] = x;
   sync();
-  double before = x - v;
   for (int w = 0; w < warp; ++w) before += red[w];
   sync();
   return before;
@@ -160,16 +163,27 @@ __device__ __forceinline__ void bitonic_sort_256(uint64_t* keys, int tid) {
   for (int e = 0; e < E; ++e) keys[tid * E + e] = v[e];
 }
 
-// The cut of one row of block scores (candidates 0..n-1, diagonal r), computed
-// by a group of NT threads: bitonic sort of 64-bit keys (descending-score rank,
-// then index) in shared memory, i.e. descending score, ascending index; then the
-// cut position of the rule: the first prefix whose fp64 cumulative sum reaches t
-// (threshold), floor(t) (Top-K) or ceil(t * n) (ratio), clamped to [1, n]. keys
-// holds P entries, P = next power of two >= n. The result is valid in thread 0
-// of the group.
+// Number of candidates kept by the Top-K / ratio rules (and by a threshold that
+// keeps everything): floor(t) (Top-K) or ceil(t * n) (ratio), in fp64 from the
+// fp32 parameter, clamped to [1, n]; NaN keeps n.
+__device__ __forceinline__ int select_rule_count(int rule, float t, int n) {
+  if (rule == kSelThreshold) return n;
+  double kk = rule == kSelTopK ? floor((double)t) : ceil((double)t * (double)n);
+  kk = kk < 1.0 ? 1.0 : (kk > (double)n ? (double)n : kk);   // NaN -> n
+  return (kk >= 1.0 && kk <= (double)n) ? (int)kk : n;
+}
+
+// The cut of one row by a full sort (rows holding a negative, infinite or NaN
+// score; select_row_cut below handles every other row without sorting):
+// bitonic sort of 64-bit keys (descending-score rank, then index) in shared
+// memory, i.e. descending score, ascending index; then the cut position of the
+// rule: the first prefix whose fp64 cumulative sum reaches t (threshold), or
+// select_rule_count. keys holds P entries, P = next power of two >= n. The
+// result is valid in thread 0 of the group.
 template <int NT, typename Sync>
-__device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, float t, int rule,
-                                 uint64_t* keys, double* red, int* first_hit, int tid, Sync sync) {
+__device__ SelCut select_row_cut_sorted(const float* __restrict__ srow, int n, int r, float t,
+                                        int rule, uint64_t* keys, double* red, int* first_hit,
+                                        int tid, Sync sync) {
   int P = 1;
   while (P < n) P <<= 1;
   for (int i = tid; i < P; i += NT)
@@ -211,11 +225,7 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
 
   if (rule != kSelThreshold) {
     // Top-K / ratio: the cut position follows from the candidate count alone
-    if (tid == 0) {
-      double kk = rule == kSelTopK ? floor((double)t) : ceil((double)t * (double)n);
-      kk = kk < 1.0 ? 1.0 : (kk > (double)n ? (double)n : kk);   // NaN -> n
-      *first_hit = (kk >= 1.0 && kk <= (double)n) ? (int)kk - 1 : n - 1;
-    }
+    if (tid == 0) *first_hit = select_rule_count(rule, t, n) - 1;
     sync();
   }
   // fp64 prefix sums over contiguous per-thread segments of the sorted order
@@ -243,6 +253,239 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   return cut;
 }
 
+// Shared state of one row's cut search (select_row_cut).
+struct SelRadix {
+  unsigned long long mass[256];   // exact mass of each bin, in units of 2^(e0 - 150)
+  int count[256];                 // candidates in each bin
+  double wmass[8];                // per-warp totals of a bin scan (groups of <= 256 threads)
+  int wcount[8];
+  double before;                  // mass of the candidates ranked before the prefix
+  int before_cnt;                 // and their number
+  int bin, last_bin;              // crossing bin of the pass; last non-empty bin
+  int bin_count;                  // candidates in the crossing bin
+  int e0;                         // exponent base of the masses (fixed by the first pass)
+  int special;                    // the row holds a negative, infinite or NaN score
+  int pick;                       // candidate index of the cut
+  SelCut sorted_cut;              // the cut of a row that went to the full sort
+};
+
+// A finite non-negative fp32 score from its descending rank (desc_rank): its
+// value is sig * 2^(e - 150) with a 24-bit integer sig and e >= 1.
+__device__ __forceinline__ void rank_sig_exp(uint32_t rk, uint32_t& sig, int& e) {
+  const uint32_t u = (~rk) & 0x7FFFFFFFu;
+  const int E = (int)(u >> 23);
+  sig = E ? ((u & 0x7FFFFFu) | 0x800000u) : (u & 0x7FFFFFu);
+  e = E ? E : 1;
+}
+
+// The cut of one row of block scores (candidates 0..n-1, diagonal r) by a
+// group of NT threads (NT a multiple of 32, at most 256), without sorting: a
+// radix search over the 32-bit descending-score ranks, eight bits per pass from
+// the top. A pass builds a 256-bin histogram of the candidates that share the
+// prefix found so far, with each bin's count and its exact mass (the scores are
+// added as integers, sig << (e - e0): every candidate left after the first pass
+// has one of two neighbouring exponents), scans the bins in rank order in fp64
+// (mass before the prefix + bins so far) and takes the first bin that reaches
+// the target: the cumulative mass t (threshold) or the kept count of the Top-K /
+// ratio rule. A bin holding one candidate ends the search; after four passes the
+// remaining candidates share one score, and the cut falls inside that tie group
+// (in index order, by adding the score in fp64 until t is reached). The result
+// is the same (score, index) cut as taking the shortest prefix of the
+// descending order (ties to the smaller index) whose cumulative mass reaches t
+// (XAttention summary, Approach; FlexPrefill rebuttal, R Q3), up to the fp64
+// rounding of the cumulative sums. A threshold t >= 1 (or NaN), or one that the
+// whole row does not reach, keeps every candidate. Rows holding a negative,
+// infinite or NaN score go to select_row_cut_sorted. `keys` holds P 64-bit
+// entries (P = next power of two >= n); its first n 32-bit words hold the ranks.
+// The result is valid in every thread of the group.
+template <int NT, typename Sync>
+__device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, float t, int rule,
+                                 uint64_t* keys, double* red, int* first_hit, SelRadix* st,
+                                 int tid, Sync sync) {
+  static_assert(NT % 32 == 0 && NT <= 256 && 256 % NT == 0, "group of 32..256 threads");
+  constexpr int BPT = 256 / NT;                 // bins per thread in a scan
+  uint32_t* ranks = reinterpret_cast<uint32_t*>(keys);
+  const int lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    st->special = 0;
+    st->before = 0.0;
+    st->before_cnt = 0;
+  }
+  sync();
+  bool special = false;
+  for (int i = tid; i < n; i += NT) {
+    const float s = srow[i];
+    const uint32_t rk = desc_rank(s);
+    special |= (rk & 0x80000000u) != 0 || !(s <= 3.4028234663852886e38f);   // negative, inf, NaN
+    ranks[i] = rk;
+  }
+  if (special) st->special = 1;
+  sync();
+  if (st->special) {
+    SelCut cut = select_row_cut_sorted<NT>(srow, n, r, t, rule, keys, red, first_hit, tid, sync);
+    if (tid == 0) st->sorted_cut = cut;   // valid in thread 0: hand it to the group
+    sync();
+    cut = st->sorted_cut;
+    sync();
+    return cut;
+  }
+
+  // target: cumulative mass t (threshold rule, t < 1) or a kept count
+  bool by_mass = rule == kSelThreshold && t < 1.0f;
+  int K = select_rule_count(rule, t, n);
+  uint32_t prefix = 0;
+  int e0 = 0;
+  bool found = false;
+  for (int pass = 0; pass < 4 && !found; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = tid; b < 256; b += NT) {
+      st->mass[b] = 0ull;
+      st->count[b] = 0;
+    }
+    if (tid == 0) { st->bin = 0x7fffffff; st->last_bin = -1; }
+    sync();
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + tid;
+      const uint32_t rk = i < n ? ranks[i] : 0u;
+      const bool valid = i < n && (pass == 0 || (rk >> (shift + 8)) == prefix);
+      const int bin = (int)((rk >> shift) & 255u);
+      uint32_t contrib = 0;
+      if (by_mass && valid) {
+        uint32_t sig;
+        int e;
+        rank_sig_exp(rk, sig, e);
+        contrib = sig << (e - (pass == 0 ? 2 * (127 - bin) : e0));
+      }
+      // one atomic per group of lanes that share a bin
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? (unsigned)bin : 256u + lane);
+      if (valid) {
+        const unsigned msum = by_mass ? __reduce_add_sync(peers, contrib) : 0u;
+        if (lane == __ffs(peers) - 1) {
+          atomicAdd(&st->count[bin], __popc(peers));
+          if (by_mass) atomicAdd(&st->mass[bin], (unsigned long long)msum);
+        }
+      }
+    }
+    sync();
+    // scan of the bins in rank order: thread tid owns bins tid*BPT .. tid*BPT+BPT-1
+    double lm[BPT];
+    int lc[BPT];
+    double tm = 0.0;
+    int tc = 0;
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) {
+      const int b = tid * BPT + k;
+      lc[k] = st->count[b];
+      lm[k] = (by_mass && lc[k]) ? ldexp((double)st->mass[b], (pass == 0 ? 2 * (127 - b) : e0) - 150)
+                                 : 0.0;
+      tm += lm[k];
+      tc += lc[k];
+      if (lc[k]) atomicMax(&st->last_bin, b);
+    }
+    double xm = tm;
+    int xc = tc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double ym = __shfl_up_sync(0xffffffffu, xm, o);
+      const int yc = __shfl_up_sync(0xffffffffu, xc, o);
+      if (lane >= o) { xm += ym; xc += yc; }
+    }
+    if (lane == 31) { st->wmass[warp] = xm; st->wcount[warp] = xc; }
+    sync();
+    double run = xm - tm;
+    int runc = xc - tc;
+    for (int w2 = 0; w2 < warp; ++w2) { run += st->wmass[w2]; runc += st->wcount[w2]; }
+    const double before = st->before;
+    const int before_cnt = st->before_cnt;
+    if (pass == 0 && by_mass) {
+      // a threshold the whole row does not reach keeps every candidate
+      double total = 0.0;
+      for (int w2 = 0; w2 < NT / 32; ++w2) total += st->wmass[w2];
+      if (!(total >= (double)t)) { by_mass = false; K = n; }
+    }
+    double excl_m = run;
+    int excl_c = runc;
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) {
+      const double incl_m = excl_m + lm[k];
+      const int incl_c = excl_c + lc[k];
+      const bool hit = lc[k] > 0 && (by_mass ? before + incl_m >= (double)t
+                                             : before_cnt + incl_c >= K);
+      if (hit) atomicMin(&st->bin, tid * BPT + k);
+      excl_m = incl_m;
+      excl_c = incl_c;
+    }
+    sync();
+    // rounding may leave the bin sums just short of what the previous pass saw:
+    // the crossing then lies in the last non-empty bin
+    const int b = st->bin != 0x7fffffff ? st->bin : st->last_bin;
+    if (b / BPT == tid) {
+      double em = run;
+      int ec = runc;
+      for (int k = 0; k < b % BPT; ++k) { em += lm[k]; ec += lc[k]; }
+      st->before = before + em;
+      st->before_cnt = before_cnt + ec;
+      st->bin_count = lc[b % BPT];
+      if (pass == 0) st->e0 = 2 * (127 - b);
+    }
+    sync();
+    if (pass == 0) e0 = st->e0;
+    prefix = (pass == 0) ? (uint32_t)b : ((prefix << 8) | (uint32_t)b);
+    if (st->bin_count == 1) {
+      // a single candidate in the crossing bin: it is the cut
+      for (int i = tid; i < n; i += NT)
+        if ((ranks[i] >> shift) == prefix) st->pick = i;
+      found = true;
+    }
+    sync();
+  }
+  int j = 1;   // position of the cut inside the tie group (1-based)
+  if (!found) {
+    // four passes: `prefix` is one exact score shared by bin_count candidates,
+    // taken in ascending index order
+    const int cnt = st->bin_count;
+    if (by_mass) {
+      const double sv = (double)rank_score(prefix);
+      double cum = st->before;
+      j = cnt;
+      for (int q = 1; q <= cnt; ++q) {
+        cum += sv;
+        if (cum >= (double)t) { j = q; break; }
+      }
+    } else {
+      j = K - st->before_cnt;
+      j = j < 1 ? 1 : (j > cnt ? cnt : j);
+    }
+    // the j-th smallest index among the tie group: contiguous segments per thread
+    const int per = (n + NT - 1) / NT;
+    const int lo = tid * per, hi = min(n, lo + per);
+    int mine = 0;
+    for (int i = lo; i < hi; ++i) mine += ranks[i] == prefix ? 1 : 0;
+    int xs = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, xs, o);
+      if (lane >= o) xs += y;
+    }
+    if (lane == 31) st->wcount[warp] = xs;
+    sync();
+    int seen = xs - mine;
+    for (int w2 = 0; w2 < warp; ++w2) seen += st->wcount[w2];
+    if (seen < j && seen + mine >= j) {
+      for (int i = lo; i < hi; ++i)
+        if (ranks[i] == prefix && ++seen == j) { st->pick = i; break; }
+    }
+    sync();
+  }
+  SelCut cut;
+  cut.index = st->pick;
+  cut.score = rank_score(ranks[cut.index]);
+  const bool diag_kept = r == cut.index || ranks_before(srow[r], r, cut.score, cut.index);
+  cut.count = st->before_cnt + (found ? 1 : j) + (diag_kept ? 0 : 1);
+  sync();   // ranks and the search state may be reused by the caller's next row
+  return cut;
+}
+
 // block c of row r is kept under the row's cut (the diagonal always is)
 __device__ __forceinline__ bool kept_by_cut(float s, int c, int r, const SelCut& cut) {
   return c == r || ranks_before(s, c, cut.score, cut.index) || (s == cut.score && c == cut.index);
@@ -254,14 +497,13 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ double red[kSelThreads / 32];
   __shared__ int first_hit;
+  __shared__ SelRadix st;
   const int row = blockIdx.x;
   const int bh = row / nb, r = row % nb, h = bh % Hq;
   const int n = causal ? r + 1 : nb;
-  int P = 1;
-  while (P < n) P <<= 1;
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
   const SelCut cut = select_row_cut<kSelThreads>(scores + (size_t)row * nb, n, r, tau[h], rule,
-                                                 keys, red, &first_hit, (int)threadIdx.x,
+                                                 keys, red, &first_hit, &st, (int)threadIdx.x,
                                                  [] { __syncthreads(); });
   if (threadIdx.x == 0) cuts[row] = cut;
 }

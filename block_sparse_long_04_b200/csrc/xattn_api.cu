@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include "attn_pair.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "score_tc.cuh"
@@ -115,29 +116,70 @@ struct FusedSelect {
   SelCut* cuts = nullptr;
 };
 
-template <int C, int G, bool SELECT>
-int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
-                    int diagonal, float scale, float* scores, float* part, float* lse_ws,
-                    FusedSelect fs, cudaStream_t st) {
-#ifndef XATTN_SCORE_BN
-#define XATTN_SCORE_BN 256
+// Scoring launches as CTA pairs (cta_group::2) by default; building with
+// XATTN_SCORE_PAIR=0 gives the single-CTA kernel.
+#ifndef XATTN_SCORE_PAIR
+#define XATTN_SCORE_PAIR 1
 #endif
-  constexpr int BN = XATTN_SCORE_BN;
-  auto kern = score_tc_kernel<C, G, BN, SELECT>;
-  constexpr int smem = ScoreTc<BN>::kSmem;
+
+template <int C, int G, bool SELECT, int PAIR>
+int launch_score_tc_mode(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
+                         int diagonal, float scale, float* scores, float* part, float* lse_ws,
+                         FusedSelect fs, cudaStream_t st) {
+  constexpr int BN = 256;
+  using L = ScoreTc<BN, PAIR>;
+  auto kern = score_tc_kernel<C, G, BN, SELECT, PAIR>;
+  constexpr int smem = L::kSmem;
   static unsigned long long done = 0;
   if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
   const int S = 128 / G;
   const int rp = M / S;
+  const int RT = (rp + 127) / 128;
   CUtensorMap mq, mk;
   if (!make_tile_map(&mq, Q, (uint64_t)B * Hq * rp, S * C, 128) ||
-      !make_tile_map(&mk, K, (uint64_t)B * Hkv * rp, S * C, BN))
+      !make_tile_map(&mk, K, (uint64_t)B * Hkv * rp, S * C, L::kKRows))
     return XATTN_ECUDA;
-  dim3 grid((rp + 127) / 128, B * Hq);
-  kern<<<grid, kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, diagonal,
-                                            scale * kLog2e, part, lse_ws, scores, fs.param,
-                                            fs.rule, fs.cuts);
+  const float sl2 = scale * kLog2e;
+  if (PAIR == 0) {
+    kern<<<dim3(RT, B * Hq), kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, diagonal,
+                                                         sl2, part, lse_ws, scores, fs.param,
+                                                         fs.rule, fs.cuts);
+    return launch_status();
+  }
+  // pairs of heads: grid (2 * RT, B*Hq/2); pairs of row tiles: (2 * ceil(RT/2), B*Hq)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = PAIR == 1 ? dim3(2 * RT, B * Hq / 2) : dim3(2 * ((RT + 1) / 2), B * Hq);
+  cfg.blockDim = dim3(kScoreTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, Hq, Hkv, M, causal, diagonal, sl2, part, lse_ws,
+                         scores, fs.param, fs.rule, fs.cuts) != cudaSuccess)
+    return XATTN_ECUDA;
   return launch_status();
+}
+
+template <int C, int G, bool SELECT>
+int launch_score_tc(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, int M, int causal,
+                    int diagonal, float scale, float* scores, float* part, float* lse_ws,
+                    FusedSelect fs, cudaStream_t st) {
+#if XATTN_SCORE_PAIR
+  // two query heads of one KV group share every key tile; otherwise two row tiles
+  if ((Hq / Hkv) % 2 == 0)
+    return launch_score_tc_mode<C, G, SELECT, 1>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale,
+                                                 scores, part, lse_ws, fs, st);
+  return launch_score_tc_mode<C, G, SELECT, 2>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale,
+                                               scores, part, lse_ws, fs, st);
+#else
+  return launch_score_tc_mode<C, G, SELECT, 0>(Q, K, B, Hq, Hkv, M, causal, diagonal, scale,
+                                               scores, part, lse_ws, fs, st);
+#endif
 }
 
 template <int C, bool SELECT>
@@ -156,10 +198,54 @@ int launch_score_c(int stride, const bf16* Q, const bf16* K, int B, int Hq, int 
   return XATTN_EUNSUPPORTED;
 }
 
+// Attention at C = 128 launches as CTA pairs (cta_group::2) by default; building
+// with XATTN_ATTN_PAIR=0 gives the single-CTA kernel everywhere.
+#ifndef XATTN_ATTN_PAIR
+#define XATTN_ATTN_PAIR 0
+#endif
+
+template <bool DENSE>
+int launch_attn_pair(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
+                     const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal,
+                     int group_rows, float scale, bf16* O, float* lse, cudaStream_t st) {
+  using L = AttnPair;
+  auto kern = attn_pair_kernel<DENSE>;
+  constexpr int smem = L::kSmem;
+  static unsigned long long done = 0;
+  if (ensure_smem_limit(kern, smem, &done) != XATTN_OK) return XATTN_ECUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_tile_map(&mq, Q, (uint64_t)B * Hq * M, L::C, 128) ||
+      !make_tile_map(&mk, K, (uint64_t)B * Hkv * M, L::C, 64) ||
+      !make_tile_map(&mv, V, (uint64_t)B * Hkv * M, L::C, 128))
+    return XATTN_ECUDA;
+  const int nb = M / 128;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ((nb + 1) / 2), B * Hq);
+  cfg.blockDim = dim3(kAttnTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, row_ptr, col_idx, Hq, Hkv, M, causal,
+                         group_rows, scale * kLog2e, O, lse) != cudaSuccess)
+    return XATTN_ECUDA;
+  return launch_status();
+}
+
 template <int C, bool DENSE>
 int launch_attn_tc(const bf16* Q, const bf16* K, const bf16* V, const int32_t* row_ptr,
                    const int32_t* col_idx, int B, int Hq, int Hkv, int M, int causal,
                    int group_rows, float scale, bf16* O, float* lse, cudaStream_t st) {
+#if XATTN_ATTN_PAIR
+  if (C == 128)
+    return launch_attn_pair<DENSE>(Q, K, V, row_ptr, col_idx, B, Hq, Hkv, M, causal, group_rows,
+                                   scale, O, lse, st);
+#endif
   auto kern = attn_tc_kernel<C, DENSE>;
   constexpr int smem = AttnTc<C>::kSmem;
   static unsigned long long done = 0;

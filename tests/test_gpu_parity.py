@@ -145,6 +145,45 @@ def test_selection_special_taus_and_ties():
     assert nnz == nb * nb + sum(len({0, r}) for r in range(nb))
 
 
+def test_selection_cut_inside_a_tie_group():
+    """Every candidate has the same score: the cut falls inside one tie group
+    (the radix search resolves all 32 rank bits, then counts in index order)."""
+    for nb, causal in ((64, False), (300, True)):
+        s = np.full((1, 3, nb, nb), 1.0, np.float64)
+        if causal:
+            s = np.tril(s)
+        s /= s.sum(-1, keepdims=True)
+        s = s.astype(np.float32)
+        tau = np.array([0.51, 0.26, 0.999], np.float32)
+        row_ptr, col, nnz = _run_select(s, tau, causal)
+        for h in range(3):
+            for r in range(nb):
+                got = col[row_ptr[h * nb + r]:row_ptr[h * nb + r + 1]]
+                want = orc.select_row(s[0, h, r].astype(np.float64), r, float(tau[h]), causal)
+                assert got.tolist() == want.tolist(), (nb, h, r)
+
+
+def test_selection_rows_with_negative_and_infinite_scores():
+    """Rows holding a negative or an infinite score (never produced by the scoring
+    kernel) take the full-sort path; the threshold and Top-K rules still follow
+    the descending order exactly."""
+    rng = np.random.default_rng(3)
+    nb, Hq = 40, 2
+    s = rng.gamma(0.5, size=(1, Hq, nb, nb))
+    s /= s.sum(-1, keepdims=True)
+    s[0, 0, 5, [1, 7, 30]] = [-0.25, -0.5, -0.125]      # negative entries
+    s[0, 1, 9, 3] = np.inf                               # an infinite entry
+    s[0, 1, 11, :] = -s[0, 1, 11, :]                     # a row of negatives only
+    s = s.astype(np.float32)
+    tau = np.array([0.6, 0.8], np.float32)
+    row_ptr, col, nnz = _run_select(s, tau, False)
+    for h in range(Hq):
+        for r in range(nb):
+            got = col[row_ptr[h * nb + r]:row_ptr[h * nb + r + 1]]
+            want = orc.select_row(s[0, h, r].astype(np.float64), r, float(tau[h]), False)
+            assert got.tolist() == want.tolist(), (h, r, got, want)
+
+
 def test_selection_capacity_error_is_reported():
     nb = 32
     s = np.tril(np.ones((1, 1, nb, nb), np.float32))
@@ -204,8 +243,12 @@ def test_dense_attention_matches_oracle(M, C, Hq, Hkv, causal):
         np.testing.assert_allclose(lse.cpu().numpy()[0, h], l, rtol=1e-4, atol=1e-4)
 
 
-def test_attention_skips_invalid_entries_and_empty_rows():
-    M, C, Hq = 512, 64, 1
+@pytest.mark.parametrize("C", [64, 128])
+def test_attention_skips_invalid_entries_and_empty_rows(C):
+    """Invalid entries are skipped, an empty row gives O = 0 and lse = -inf. At
+    C = 128 the query blocks run in pairs over the union of their lists, so this
+    also covers a pair whose two lists are empty / disjoint / nested."""
+    M, Hq = 512, 1
     w = small_workload(M, C, Hq, 1, 8, True)
     (Qb, Kb, Vb), (Q, K, V) = device_inputs(w)
     nb = 4
