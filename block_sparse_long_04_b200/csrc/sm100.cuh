@@ -206,10 +206,13 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release;\n barrier.cluster.wait.acquire;" ::: "memory");
 }
-// arrive on an mbarrier given by its shared::cluster address (possibly the peer's)
+// arrive on an mbarrier given by its shared::cluster address (possibly the
+// peer's), with the default (CTA-scope release) semantics: what the arrival
+// publishes is tensor-memory state, which tcgen05.wait / tcgen05.fence order; a
+// cluster-scope release would make every arriving thread wait for a cluster-wide
+// memory fence
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                   bar_cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 // 2-D tiled load into this CTA's shared memory whose completion (bytes) is counted
 // on an mbarrier that may live in the peer CTA (its shared::cluster address): the
