@@ -269,6 +269,11 @@ struct SelRadix {
   SelCut sorted_cut;              // the cut of a row that went to the full sort
 };
 
+// 2^k for an integer k in the normal fp64 range, exactly
+__device__ __forceinline__ double pow2_f64(int k) {
+  return __longlong_as_double((long long)(k + 1023) << 52);
+}
+
 // A finite non-negative fp32 score from its descending rank (desc_rank): its
 // value is sig * 2^(e - 150) with a 24-bit integer sig and e >= 1.
 __device__ __forceinline__ void rank_sig_exp(uint32_t rk, uint32_t& sig, int& e) {
@@ -376,8 +381,9 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
     for (int k = 0; k < BPT; ++k) {
       const int b = tid * BPT + k;
       lc[k] = st->count[b];
-      lm[k] = (by_mass && lc[k]) ? ldexp((double)st->mass[b], (pass == 0 ? 2 * (127 - b) : e0) - 150)
-                                 : 0.0;
+      lm[k] = (by_mass && lc[k])
+                  ? (double)st->mass[b] * pow2_f64((pass == 0 ? 2 * (127 - b) : e0) - 150)
+                  : 0.0;
       tm += lm[k];
       tc += lc[k];
       if (lc[k]) atomicMax(&st->last_bin, b);
@@ -491,22 +497,37 @@ __device__ __forceinline__ bool kept_by_cut(float s, int c, int r, const SelCut&
   return c == r || ranks_before(s, c, cut.score, cut.index) || (s == cut.score && c == cut.index);
 }
 
+// One CTA of kSelThreads threads holds RPC rows, a group of NT = kSelThreads /
+// RPC threads per row with its own named barrier; `keys` (dynamic shared
+// memory) holds P 64-bit entries per group. Short rows run four to a CTA (64
+// threads each): the cut search's fixed cost per pass is paid by fewer threads.
+template <int RPC>
 __global__ void __launch_bounds__(kSelThreads)
 select_count_kernel(const float* __restrict__ scores, const float* __restrict__ tau, int Hq, int nb,
-                    int causal, SelCut* __restrict__ cuts, int rule) {
+                    int causal, SelCut* __restrict__ cuts, int rule, int rows, int P) {
+  constexpr int NT = kSelThreads / RPC;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ double red[kSelThreads / 32];
-  __shared__ int first_hit;
-  __shared__ SelRadix st;
-  const int row = blockIdx.x;
+  __shared__ double red[RPC][NT / 32];
+  __shared__ int first_hit[RPC];
+  __shared__ SelRadix st[RPC];
+  const int grp = (int)threadIdx.x / NT, tid = (int)threadIdx.x % NT;
+  const int row = blockIdx.x * RPC + grp;
+  if (row >= rows) return;   // whole groups leave; the others sync on their own barriers
   const int bh = row / nb, r = row % nb, h = bh % Hq;
   const int n = causal ? r + 1 : nb;
-  uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
-  const SelCut cut = select_row_cut<kSelThreads>(scores + (size_t)row * nb, n, r, tau[h], rule,
-                                                 keys, red, &first_hit, &st, (int)threadIdx.x,
-                                                 [] { __syncthreads(); });
-  if (threadIdx.x == 0) cuts[row] = cut;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + (size_t)grp * P;
+  const int bar = 1 + grp;
+  auto sync = [bar] {
+    if (RPC == 1) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(bar), "n"(NT) : "memory");
+  };
+  const SelCut cut = select_row_cut<NT>(scores + (size_t)row * nb, n, r, tau[h], rule, keys,
+                                        red[grp], &first_hit[grp], &st[grp], tid, sync);
+  if (tid == 0) cuts[row] = cut;
 }
+
+// Rows of at most this many candidates run four to a CTA.
+constexpr int kSelShortRow = 2048;
 
 __global__ void __launch_bounds__(1024)
 select_scan_kernel(const SelCut* __restrict__ cuts, int rows, int32_t* __restrict__ row_ptr,

@@ -368,6 +368,28 @@ size_t xattn_select_workspace_size(int B, int Hq, int nb) {
   return (bytes + 255) & ~(size_t)255;
 }
 
+// The count pass of the selection: rows of at most kSelShortRow candidates four
+// to a CTA (64 threads each), longer rows one to a CTA.
+static int launch_select_count(const float* scores, const float* param, int Hq, int nb, int causal,
+                               SelCut* cuts, int rule, long long rows, cudaStream_t st) {
+  int P = 1;
+  while (P < nb) P <<= 1;
+  if (P <= kSelShortRow) {
+    static unsigned long long done = 0;
+    if (ensure_smem_limit(select_count_kernel<4>, 4 * kSelShortRow * 8, &done) != XATTN_OK)
+      return XATTN_ECUDA;
+    select_count_kernel<4><<<(unsigned)((rows + 3) / 4), kSelThreads, 4 * P * 8, st>>>(
+        scores, param, Hq, nb, causal ? 1 : 0, cuts, rule, (int)rows, P);
+  } else {
+    static unsigned long long done = 0;
+    if (ensure_smem_limit(select_count_kernel<1>, kSelMaxNb * 8, &done) != XATTN_OK)
+      return XATTN_ECUDA;
+    select_count_kernel<1><<<(unsigned)rows, kSelThreads, P * 8, st>>>(
+        scores, param, Hq, nb, causal ? 1 : 0, cuts, rule, (int)rows, P);
+  }
+  return cudaGetLastError() == cudaSuccess ? XATTN_OK : XATTN_ECUDA;
+}
+
 // Checks and launches of the per-head selection (count, scan, fill) with the
 // per-row scratch `cuts` supplied by the caller of this helper: the workspace of
 // xattn_select / xattn_select_ex, or the library's fixed array for
@@ -384,12 +406,8 @@ static int select_launch(const float* scores, const float* param, int rule, int 
   }
   if (!scores || !param || !col_idx) return XATTN_EINVAL;
   if (cuts == nullptr) return XATTN_ECUDA;
-  int P = 1;
-  while (P < nb) P <<= 1;
-  static unsigned long long done = 0;
-  if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
-  select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, param, Hq, nb,
-                                                                  causal ? 1 : 0, cuts, rule);
+  if (launch_select_count(scores, param, Hq, nb, causal, cuts, rule, rows, st) != XATTN_OK)
+    return XATTN_ECUDA;
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
   const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
   select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
@@ -471,12 +489,8 @@ int xattn_select_group(const float* scores, const float* param, int rule, int B,
   SelCut* cuts = static_cast<SelCut*>(workspace);
   SelCut* gcuts = reinterpret_cast<SelCut*>(static_cast<uint8_t*>(workspace) +
                                             xattn_select_workspace_size(B, Hq, nb));
-  int P = 1;
-  while (P < nb) P <<= 1;
-  static unsigned long long done = 0;
-  if (ensure_smem_limit(select_count_kernel, kSelMaxNb * 8, &done) != XATTN_OK) return XATTN_ECUDA;
-  select_count_kernel<<<(unsigned)rows, kSelThreads, P * 8, st>>>(scores, param, Hq, nb,
-                                                                  causal ? 1 : 0, cuts, rule);
+  if (launch_select_count(scores, param, Hq, nb, causal, cuts, rule, rows, st) != XATTN_OK)
+    return XATTN_ECUDA;
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
   select_group_count_kernel<<<(unsigned)grows, kSelThreads, 0, st>>>(scores, cuts, Hq, Hkv, nb,
                                                                      causal ? 1 : 0, gcuts);
