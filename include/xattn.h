@@ -265,7 +265,9 @@ XATTN_API int xattn_select_noalloc(const float* scores, const float* tau, int B,
  *   Q, O       bf16 [B, Hq, M, C];  K, V  bf16 [B, Hkv, M, C]
  *   row_ptr, col_idx  CSR as produced by xattn_select (device memory). Entries
  *              outside [0, M/block), and entries c > r when causal, are skipped;
- *              any order is accepted. The caller guarantees that every
+ *              any order is accepted; a block listed twice is attended twice
+ *              (its keys count twice in the softmax), so lists should not repeat
+ *              an entry. The caller guarantees that every
  *              row_ptr[i] .. row_ptr[i+1] range lies inside col_idx (the
  *              kernel reads col_idx there without a bound; a row with
  *              row_ptr[i+1] <= row_ptr[i] is empty).
