@@ -332,21 +332,37 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   asm volatile("bar.sync 1, 384;" ::: "memory");
   const bool done_ok = !*abort_flag;
   if (done_ok) {
+    // each thread takes two columns at a time and issues their partial loads (up
+    // to 2 x 16) before it consumes any, so the L2 latency is paid once per batch
     const float inv_g = 1.f / (float)G;
+    constexpr int U = G < 16 ? G : 16;
     for (int k = 0; k < 128 / G; ++k) {
       const int r = i0 / G + k;
       if (r >= nb) break;
       const int ncand = causal ? r + 1 : nb;
       float* srow = scores + ((size_t)bh * nb + r) * nb;
       const float* pr0 = part + part_row<G>(bh, r * G, rp, nb, causal);
-      for (int c = tid; c < nb; c += kScoreTcThreads) {
-        float acc = 0.f;
-        if (c < ncand) {
-#pragma unroll 4
-          for (int i = 0; i < G; ++i) acc += ex2(pr0[(size_t)i * ncand + c] - lse_s[r * G + i - i0]);
-          acc *= inv_g;
+      const float* lrow = lse_s + r * G - i0;
+      for (int c0 = tid; c0 < nb; c0 += 2 * kScoreTcThreads) {
+        const int c1 = c0 + kScoreTcThreads;
+        const bool v0 = c0 < ncand, v1 = c1 < ncand;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll 1
+        for (int ib = 0; ib < G; ib += U) {
+          float x0[U], x1[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            x0[u] = v0 ? pr0[(size_t)(ib + u) * ncand + c0] : kNegInf;
+            x1[u] = v1 ? pr0[(size_t)(ib + u) * ncand + c1] : kNegInf;
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            a0 += ex2(x0[u] - lrow[ib + u]);
+            a1 += ex2(x1[u] - lrow[ib + u]);
+          }
         }
-        srow[c] = acc;
+        srow[c0] = v0 ? a0 * inv_g : 0.f;
+        if (c1 < nb) srow[c1] = v1 ? a1 * inv_g : 0.f;
       }
     }
   }
