@@ -19,7 +19,7 @@ import torch
 import oracle as orc
 import synthetic as sy
 from tests import parity as P
-from tests.gpu_util import poison_buffers, poisoned, poisoned_like, bf16_to_np, to_dev
+from tests.gpu_util import bf16_to_np, poisoned, poisoned_like, to_dev
 
 pytestmark = pytest.mark.gpu
 

@@ -14,8 +14,8 @@ import torch
 import oracle as orc
 import synthetic as sy
 from tests import parity as P
-from tests.gpu_util import (poison_buffers, poisoned, poisoned_like, bf16_to_np, csr_to_dict, device_inputs, dict_to_csr,
-                            small_workload, to_dev)
+from tests.gpu_util import (bf16_to_np, csr_to_dict, device_inputs, dict_to_csr, poison_buffers,
+                            poisoned, poisoned_like, small_workload)
 
 pytestmark = pytest.mark.gpu
 

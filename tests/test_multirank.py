@@ -3,7 +3,6 @@ is the max over ranks, the whole-job metric divides by every rank's layers, and
 the reference arm runs on rank 0 only."""
 import json
 import math
-import os
 import socket
 
 import pytest

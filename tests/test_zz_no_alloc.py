@@ -18,7 +18,7 @@ import numpy as np
 import pytest
 import torch
 
-from tests.gpu_util import poison_buffers, poisoned, poisoned_like
+from tests.gpu_util import poisoned
 
 from block_sparse_long_04_b200 import build as _build
 
