@@ -47,12 +47,16 @@ constexpr int kScoreTcThreads = 384;
 // neighbouring row tiles of one head. In a pair each CTA holds its own 128 query
 // rows and half of every BN-column key tile, so each SM reads and stores half the
 // key bytes of a single-CTA tile.
-template <int BN, int PAIR = 0>
+// NB: 64-wide boxes of the reshaped width per stage (NB = 2: 128-wide stages of
+// eight K = 16 MMAs, so that the issuing thread waits and commits once per eight).
+template <int BN, int PAIR = 0, int NB = 1>
 struct ScoreTc {
-  static constexpr int kStages = PAIR ? 6 : (BN == 256 ? 4 : 6);
-  static constexpr int kQBytes = 128 * 128;              // 128 rows x 64 bf16
+  static constexpr int kStages = (PAIR ? 6 : (BN == 256 ? 4 : 6)) / NB;
+  static constexpr int kBoxQ = 128 * 128;                // 128 rows x 64 bf16
   static constexpr int kKRows = PAIR ? BN / 2 : BN;      // key rows this CTA loads
-  static constexpr int kKBytes = kKRows * 128;           // kKRows rows x 64 bf16
+  static constexpr int kBoxK = kKRows * 128;             // kKRows rows x 64 bf16
+  static constexpr int kQBytes = NB * kBoxQ;
+  static constexpr int kKBytes = NB * kBoxK;
   static constexpr int kStageBytes = kQBytes + kKBytes;
   static constexpr int kOffBar = kStages * kStageBytes;
   static constexpr int kOffLse = kOffBar + 256;
@@ -74,18 +78,21 @@ constexpr int kSelRingRed = kSelMaxNb * 8;
 constexpr int kSelRingRadix = kSelMaxNb * 8 + 256;
 static_assert(ScoreTc<128>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix) &&
               ScoreTc<256>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix) &&
-              ScoreTc<256, 1>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix),
+              ScoreTc<256, 1>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix) &&
+              ScoreTc<256, 1, 2>::kOffBar >= kSelRingRadix + (int)sizeof(SelRadix),
               "the stage ring must hold the fused selection's keys and search state");
 
-// Offset of reshaped row ip's partial log-masses in the workspace. Non-causal:
-// nb entries per row. Causal: the g = G rows of query block r hold only the
-// r + 1 key blocks they can see, so head bh's rows are packed as a triangle of
-// G * nb * (nb + 1) / 2 = rp * (nb + 1) / 2 entries (half of the non-causal size).
+// Offset of the partial log-mass of reshaped row ip in key block c. Each key
+// block holds one run of rows: all rp of them (non-causal), or only the rows of
+// the query blocks that can see it (ip >= c * G, rp - c * G entries) when causal,
+// so that head bh takes rp * (nb + 1) / 2 entries (half of the non-causal size).
+// Rows are contiguous, so a warp's stores for one block (32 rows) are coalesced
+// and the finalize reads the G rows of a query block as one run.
 template <int G>
-__device__ __forceinline__ size_t part_row(int bh, int ip, int rp, int nb, int causal) {
-  if (!causal) return ((size_t)bh * rp + ip) * nb;
-  const size_t r = (size_t)(ip / G), i = (size_t)(ip % G);
-  return (size_t)bh * ((size_t)rp * (nb + 1) / 2) + G * (r * (r + 1) / 2) + i * (r + 1);
+__device__ __forceinline__ size_t part_at(int bh, int c, int ip, int rp, int nb, int causal) {
+  if (!causal) return ((size_t)bh * nb + c) * rp + ip;
+  return (size_t)bh * ((size_t)rp * (nb + 1) / 2) + (size_t)c * rp -
+         (size_t)G * ((size_t)c * (c + 1) / 2) + ip;
 }
 
 template <int C, int G, int BN, bool SELECT, int PAIR>
@@ -94,10 +101,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 int Hq, int Hkv, int M, int causal, int diagonal, float scale_log2,
                 float* __restrict__ part, float* __restrict__ lse_ws, float* __restrict__ scores,
                 const float* __restrict__ sel_param, int sel_rule, SelCut* __restrict__ cuts) {
-  using L = ScoreTc<BN, PAIR>;
-  constexpr int ST = L::kStages;
   constexpr int S = 128 / G;
-  constexpr int NCH = S * C / 64;       // 64-wide chunks of the reshaped width
+  constexpr int NBX = (PAIR && S * C >= 128) ? 2 : 1;   // 64-wide boxes per stage
+  using L = ScoreTc<BN, PAIR, NBX>;
+  constexpr int ST = L::kStages;
+  constexpr int NCH = S * C / (64 * NBX);   // stages per column tile
   using namespace sm100;
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -188,18 +196,26 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int st = it % ST;
         if (it >= ST && !mbar_wait(&empty[st], ((it / ST) - 1) & 1, abort_flag)) break;
         const int jt = it / NCH, q = it % NCH;
-        const int s = (q * 64) / C, d0 = (q * 64) % C;
         const uint32_t dst = sbase + st * L::kStageBytes;
-        // antidiagonal: query rows reversed inside the stride group; diagonal: forward
-        const int xq = (diagonal ? s : S - 1 - s) * C + d0;
         if (PAIR) {
           if (leader) mbar_expect_tx(&full[st], 2 * L::kStageBytes);
-          tma_load_2d_pair(dst, &tmQ, xq, yq, full_lead + st * 8);
-          tma_load_2d_pair(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, full_lead + st * 8);
         } else {
           mbar_expect_tx(&full[st], L::kStageBytes);
-          tma_load_2d(dst, &tmQ, xq, yq, &full[st]);
-          tma_load_2d(dst + L::kQBytes, &tmK, s * C + d0, yk0 + jt * BN, &full[st]);
+        }
+#pragma unroll
+        for (int h = 0; h < NBX; ++h) {
+          const int w = (q * NBX + h) * 64;          // reshaped column of the box
+          const int s = w / C, d0 = w % C;
+          // antidiagonal: query rows reversed inside the stride group; diagonal: forward
+          const int xq = (diagonal ? s : S - 1 - s) * C + d0;
+          const uint32_t dq = dst + h * L::kBoxQ, dk = dst + L::kQBytes + h * L::kBoxK;
+          if (PAIR) {
+            tma_load_2d_pair(dq, &tmQ, xq, yq, full_lead + st * 8);
+            tma_load_2d_pair(dk, &tmK, s * C + d0, yk0 + jt * BN, full_lead + st * 8);
+          } else {
+            tma_load_2d(dq, &tmQ, xq, yq, &full[st]);
+            tma_load_2d(dk, &tmK, s * C + d0, yk0 + jt * BN, &full[st]);
+          }
         }
       }
       // drain: every load issued must land before the CTA may exit (the leader's
@@ -218,25 +234,32 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // halves of the key tile) and signals both CTAs' barriers; the other CTA's
       // issuer only waits for the pair's last MMA
       if (leader) {
+        // One thread issues every MMA, so its loop is kept short: the stage's
+        // descriptors are the stage-0 descriptors plus the stage offset (the
+        // address field holds the shared address >> 4; no carry leaves it below
+        // 256 KB), and the stage, parity and tile counters advance by increments.
         constexpr uint32_t idesc = idesc_bf16_f32(PAIR ? 256 : 128, BN, false, false);
+        const uint64_t da0 = smem_desc_sw128(sbase, 16, 1024);
+        const uint64_t db0 = smem_desc_sw128(sbase + L::kQBytes, 16, 1024);
+        constexpr uint32_t kStageDesc = L::kStageBytes >> 4;
         bool ok = true;
-        for (int it = 0; ok && it < total; ++it) {
-          const int st = it % ST;
-          const int jt = it / NCH, q = it % NCH;
+        int st = 0, q = 0, jt = 0;
+        uint32_t ph = 0;
+        for (int it = 0; it < total; ++it) {
           const int buf = jt & 1;
           if (q == 0 && jt >= 2) {
-            if (!(ok = mbar_wait(&acc_empty[buf], ((jt / 2) - 1) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&acc_empty[buf], ((jt >> 1) - 1) & 1, abort_flag))) break;
           }
-          if (!(ok = mbar_wait(&full[st], (it / ST) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&full[st], ph, abort_flag))) break;
           tc_fence_after();
-          const uint32_t a0 = sbase + st * L::kStageBytes;
-          const uint32_t b0 = a0 + L::kQBytes;
+          const uint64_t da = da0 + (uint64_t)(st * kStageDesc);
+          const uint64_t db = db0 + (uint64_t)(st * kStageDesc);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t da = smem_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t db = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-            if (PAIR) mma_f16_ss_pair(tmem + buf * BN, da, db, idesc, (q > 0 || kk > 0) ? 1u : 0u);
-            else mma_f16_ss(tmem + buf * BN, da, db, idesc, (q > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4 * NBX; ++kk) {   // 16 bf16 (32 bytes) along K per MMA
+            const uint32_t oa = (kk >> 2) * (L::kBoxQ >> 4) + (kk & 3) * 2;
+            const uint32_t ob = (kk >> 2) * (L::kBoxK >> 4) + (kk & 3) * 2;
+            if (PAIR) mma_f16_ss_pair(tmem + buf * BN, da + oa, db + ob, idesc, (q | kk) ? 1u : 0u);
+            else mma_f16_ss(tmem + buf * BN, da + oa, db + ob, idesc, (q | kk) ? 1u : 0u);
           }
           if (PAIR) {
             mma_commit_pair(&empty[st]);
@@ -245,7 +268,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mma_commit(&empty[st]);
             if (q == NCH - 1) mma_commit(&acc_full[buf]);
           }
+          if (++st == ST) { st = 0; ph ^= 1u; }
+          if (++q == NCH) { q = 0; ++jt; }
         }
+        (void)ok;
         if (PAIR) mma_commit_pair(drain);
         else mma_commit(drain);
       }
@@ -260,6 +286,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int rl = (warp & 3) * 32 + lane;     // row within the tile
     const int ip = i0 + rl;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    // Each thread sums its half row against one reference m_run (log2 units), set
+    // by its first visible block and raised only when a block's maximum exceeds it
+    // by more than 2^64 (then l_run is rescaled), so a key block costs one
+    // exponential per element and one logarithm; masking is applied only to the
+    // column chunks that cross the causal diagonal or the end of the rows.
+    constexpr float kHeadroom = 64.f;
+    const float2 s2 = make_float2(scale_log2, scale_log2);
     float m_run = kNegInf, l_run = 0.f;
     bool ok = true;
     for (int jt = 0; jt < njt; ++jt) {
@@ -283,26 +316,35 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
         const int j0 = jt * BN + hh * 128 + ch * CH;
+        if ((causal && j0 + CH - 1 > ip) || j0 + CH > rp) {
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const int jp = j0 + i;
+            if (!(jp < rp && (!causal || jp <= ip))) v[i] = kNegInf;
+          }
+        }
 #pragma unroll
         for (int kb = 0; kb < CH / G; ++kb) {
-          float vmax = kNegInf;
+          const float* x = v + kb * G;
+          float bm = kNegInf;
 #pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const int jp = j0 + kb * G + i;
-            float x = v[kb * G + i] * scale_log2;
-            x = (jp < rp && (!causal || jp <= ip)) ? x : kNegInf;
-            v[kb * G + i] = x;
-            vmax = fmaxf(vmax, x);
-          }
-          if (vmax != kNegInf) {
-            float sum = 0.f;
+          for (int i = 0; i < G; i += 2) bm = fmax3(bm, x[i], x[i + 1]);
+          if (bm != kNegInf) {
+            const float bms = bm * scale_log2;
+            if (bms > m_run + kHeadroom) {   // first visible block, or growth past the headroom
+              l_run *= ex2(m_run - bms);
+              m_run = bms;
+            }
+            const float2 nm2 = make_float2(-m_run, -m_run);
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < G; ++i) sum += ex2(v[kb * G + i] - vmax);
-            const float ell = vmax + lg2(sum);
-            const float mn = fmaxf(m_run, ell);
-            l_run = l_run * ex2(m_run - mn) + ex2(ell - mn);
-            m_run = mn;
-            if (ip < rp) part[part_row<G>(bh, ip, rp, nb, causal) + (j0 / G + kb)] = ell;
+            for (int i = 0; i < G; i += 2) {
+              const float2 t2 = ffma2(make_float2(x[i], x[i + 1]), s2, nm2);
+              acc = fadd2(acc, make_float2(ex2(t2.x), ex2(t2.y)));
+            }
+            const float sum = acc.x + acc.y;
+            l_run += sum;
+            if (ip < rp) part[part_at<G>(bh, j0 / G + kb, ip, rp, nb, causal)] = m_run + lg2(sum);
           }
         }
       }
@@ -328,41 +370,75 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   // The producer and MMA warps are idle by now, so all 384 threads turn the
   // partials of the CTA's rows into block scores (a wait that failed has set
-  // the abort flag, which every thread reads after the barrier).
+  // the abort flag, which every thread reads after the barrier). Lane 0 of the
+  // producer and MMA warps ran their loops alone; each warp reconverges before
+  // the CTA barrier.
+  __syncwarp();
   asm volatile("bar.sync 1, 384;" ::: "memory");
   const bool done_ok = !*abort_flag;
   if (done_ok) {
-    // each thread takes two columns at a time and issues their partial loads (up
-    // to 2 x 16) before it consumes any, so the L2 latency is paid once per batch
+    // The (query block r, column c) items of the CTA's rows are spread over the
+    // threads: an item's G partials are one aligned run, read by G / VEC
+    // neighbouring lanes with one VEC-wide load each, so that a warp's load
+    // covers whole runs; the lanes' sums are combined by shuffles. Each thread
+    // issues the loads of R items before it consumes any, so the L2 latency is
+    // paid once per batch. Columns a causal row cannot see are written as zeros
+    // in a pass of their own.
     const float inv_g = 1.f / (float)G;
-    constexpr int U = G < 16 ? G : 16;
-    for (int k = 0; k < 128 / G; ++k) {
-      const int r = i0 / G + k;
-      if (r >= nb) break;
-      const int ncand = causal ? r + 1 : nb;
-      float* srow = scores + ((size_t)bh * nb + r) * nb;
-      const float* pr0 = part + part_row<G>(bh, r * G, rp, nb, causal);
-      const float* lrow = lse_s + r * G - i0;
-      for (int c0 = tid; c0 < nb; c0 += 2 * kScoreTcThreads) {
-        const int c1 = c0 + kScoreTcThreads;
-        const bool v0 = c0 < ncand, v1 = c1 < ncand;
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll 1
-        for (int ib = 0; ib < G; ib += U) {
-          float x0[U], x1[U];
+    constexpr int VEC = G < 4 ? G : 4;                    // partials per lane and item
+    constexpr int TPI = G / VEC;                          // lanes per item (1..32)
+    constexpr int IPR = kScoreTcThreads / TPI;            // items per round of the CTA
+    constexpr int R = 16;                                 // items per thread and batch
+    const int sub = tid % TPI, slot = tid / TPI;
+    const int rb = i0 / G;                                // first query block of the tile
+    const int KB = max(0, min(128 / G, nb - rb));         // query blocks of the tile
+    auto ncand_of = [&](int k) { return causal ? rb + k + 1 : nb; };
+    // items of query blocks < k: causal k (rb + 1) + k (k - 1) / 2, else k nb
+    auto items_before = [&](int k) {
+      return causal ? k * (rb + 1) + k * (k - 1) / 2 : k * nb;
+    };
+    const int nitems = items_before(KB);
+    int k = 0;   // query block of the thread's current item (items rise with the batch)
+    for (int b0 = 0; b0 < nitems; b0 += R * IPR) {
+      int kk[R], cc[R];
+      float x[R][VEC];
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            x0[u] = v0 ? pr0[(size_t)(ib + u) * ncand + c0] : kNegInf;
-            x1[u] = v1 ? pr0[(size_t)(ib + u) * ncand + c1] : kNegInf;
-          }
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            a0 += ex2(x0[u] - lrow[ib + u]);
-            a1 += ex2(x1[u] - lrow[ib + u]);
-          }
+      for (int j = 0; j < R; ++j) {
+        const int item = b0 + j * IPR + slot;
+        while (k + 1 < KB && item >= items_before(k + 1)) ++k;
+        kk[j] = item < nitems ? k : -1;
+        cc[j] = item - items_before(k);
+        // the run starts at a multiple of G floats and this lane's part at a
+        // multiple of VEC: 16-byte (VEC = 4) or 8-byte (VEC = 2) aligned
+        const float* pr = part + part_at<G>(bh, kk[j] < 0 ? 0 : cc[j],
+                                            (rb + (kk[j] < 0 ? 0 : k)) * G + sub * VEC, rp, nb,
+                                            causal);
+        if constexpr (VEC == 4) {
+          const float4 t4 = kk[j] >= 0 ? *reinterpret_cast<const float4*>(pr)
+                                       : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
+          x[j][0] = t4.x; x[j][1] = t4.y; x[j][2] = t4.z; x[j][3] = t4.w;
+        } else {
+          const float2 t2 = kk[j] >= 0 ? *reinterpret_cast<const float2*>(pr)
+                                       : make_float2(kNegInf, kNegInf);
+          x[j][0] = t2.x; x[j][1] = t2.y;
         }
-        srow[c0] = v0 ? a0 * inv_g : 0.f;
-        if (c1 < nb) srow[c1] = v1 ? a1 * inv_g : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const float* lrow = lse_s + (kk[j] < 0 ? 0 : kk[j]) * G + sub * VEC;
+        float a = 0.f;
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) a += kk[j] >= 0 ? ex2(x[j][u] - lrow[u]) : 0.f;
+#pragma unroll
+        for (int o = TPI / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (sub == 0 && kk[j] >= 0)
+          scores[((size_t)bh * nb + rb + kk[j]) * nb + cc[j]] = a * inv_g;
+      }
+    }
+    if (causal) {
+      for (int k2 = 0; k2 < KB; ++k2) {
+        float* srow = scores + ((size_t)bh * nb + rb + k2) * nb;
+        for (int c = ncand_of(k2) + tid; c < nb; c += kScoreTcThreads) srow[c] = 0.f;
       }
     }
   }

@@ -127,7 +127,7 @@ int launch_score_tc_mode(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, i
                          int diagonal, float scale, float* scores, float* part, float* lse_ws,
                          FusedSelect fs, cudaStream_t st) {
   constexpr int BN = 256;
-  using L = ScoreTc<BN, PAIR>;
+  using L = ScoreTc<BN, PAIR, (PAIR && (128 / G) * C >= 128) ? 2 : 1>;   // the kernel's layout
   auto kern = score_tc_kernel<C, G, BN, SELECT, PAIR>;
   constexpr int smem = L::kSmem;
   static unsigned long long done = 0;
