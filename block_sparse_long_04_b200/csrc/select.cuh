@@ -255,7 +255,11 @@ __device__ SelCut select_row_cut_sorted(const float* __restrict__ srow, int n, i
 
 // Shared state of one row's cut search (select_row_cut).
 struct SelRadix {
-  unsigned long long mass[256];   // exact mass of each bin, in units of 2^(e0 - 150)
+  // exact mass of each bin, in units of 2^(e0 - 150): mass_hi * 2^16 + mass_lo,
+  // kept as two 32-bit sums so that every update is a native 32-bit atomic (a
+  // candidate adds at most 2^25, a row holds at most kSelMaxNb = 2^13 of them)
+  unsigned mass_lo[256];
+  unsigned mass_hi[256];
   int count[256];                 // candidates in each bin
   double wmass[8];                // per-warp totals of a bin scan (groups of <= 256 threads)
   int wcount[8];
@@ -318,6 +322,7 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   }
   sync();
   bool special = false;
+#pragma unroll 4
   for (int i = tid; i < n; i += NT) {
     const float s = srow[i];
     const uint32_t rk = desc_rank(s);
@@ -344,7 +349,8 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   for (int pass = 0; pass < 4 && !found; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int b = tid; b < 256; b += NT) {
-      st->mass[b] = 0ull;
+      st->mass_lo[b] = 0u;
+      st->mass_hi[b] = 0u;
       st->count[b] = 0;
     }
     if (tid == 0) { st->bin = 0x7fffffff; st->last_bin = -1; }
@@ -361,13 +367,28 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
         rank_sig_exp(rk, sig, e);
         contrib = sig << (e - (pass == 0 ? 2 * (127 - bin) : e0));
       }
-      // one atomic per group of lanes that share a bin
-      const unsigned peers = __match_any_sync(0xffffffffu, valid ? (unsigned)bin : 256u + lane);
-      if (valid) {
-        const unsigned msum = by_mass ? __reduce_add_sync(peers, contrib) : 0u;
-        if (lane == __ffs(peers) - 1) {
-          atomicAdd(&st->count[bin], __popc(peers));
-          if (by_mass) atomicAdd(&st->mass[bin], (unsigned long long)msum);
+      if (pass == 0) {
+        // the first pass bins by exponent pairs, so a warp's candidates share a
+        // few bins: one set of atomics per group of lanes with the same bin (the
+        // match costs more the more distinct values a warp holds)
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? (unsigned)bin : 256u + lane);
+        if (valid) {
+          const unsigned mlo = by_mass ? __reduce_add_sync(peers, contrib & 0xFFFFu) : 0u;
+          const unsigned mhi = by_mass ? __reduce_add_sync(peers, contrib >> 16) : 0u;
+          if (lane == __ffs(peers) - 1) {
+            atomicAdd(&st->count[bin], __popc(peers));
+            if (by_mass) {
+              atomicAdd(&st->mass_lo[bin], mlo);
+              atomicAdd(&st->mass_hi[bin], mhi);
+            }
+          }
+        }
+      } else if (valid) {
+        // later passes spread a warp's candidates over many bins: plain atomics
+        atomicAdd(&st->count[bin], 1);
+        if (by_mass) {
+          atomicAdd(&st->mass_lo[bin], contrib & 0xFFFFu);
+          atomicAdd(&st->mass_hi[bin], contrib >> 16);
         }
       }
     }
@@ -376,18 +397,22 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
     double lm[BPT];
     int lc[BPT];
     double tm = 0.0;
-    int tc = 0;
+    int tc = 0, my_last = -1;
 #pragma unroll
     for (int k = 0; k < BPT; ++k) {
       const int b = tid * BPT + k;
       lc[k] = st->count[b];
       lm[k] = (by_mass && lc[k])
-                  ? (double)st->mass[b] * pow2_f64((pass == 0 ? 2 * (127 - b) : e0) - 150)
+                  ? (double)(((unsigned long long)st->mass_hi[b] << 16) + st->mass_lo[b]) *
+                        pow2_f64((pass == 0 ? 2 * (127 - b) : e0) - 150)
                   : 0.0;
       tm += lm[k];
       tc += lc[k];
-      if (lc[k]) atomicMax(&st->last_bin, b);
+      if (lc[k]) my_last = b;
     }
+    // one shared atomic per warp: the last non-empty bin
+    my_last = __reduce_max_sync(0xffffffffu, my_last);
+    if (lane == 0 && my_last >= 0) atomicMax(&st->last_bin, my_last);
     double xm = tm;
     int xc = tc;
 #pragma unroll
@@ -411,16 +436,20 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
     }
     double excl_m = run;
     int excl_c = runc;
+    int my_hit = 0x7fffffff;   // this thread's first bin that reaches the target
 #pragma unroll
     for (int k = 0; k < BPT; ++k) {
       const double incl_m = excl_m + lm[k];
       const int incl_c = excl_c + lc[k];
       const bool hit = lc[k] > 0 && (by_mass ? before + incl_m >= (double)t
                                              : before_cnt + incl_c >= K);
-      if (hit) atomicMin(&st->bin, tid * BPT + k);
+      if (hit && my_hit == 0x7fffffff) my_hit = tid * BPT + k;
       excl_m = incl_m;
       excl_c = incl_c;
     }
+    // one shared atomic per warp: the first bin of the group that reaches it
+    my_hit = (int)__reduce_min_sync(0xffffffffu, (unsigned)my_hit);
+    if (lane == 0 && my_hit != 0x7fffffff) atomicMin(&st->bin, my_hit);
     sync();
     // rounding may leave the bin sums just short of what the previous pass saw:
     // the crossing then lies in the last non-empty bin
@@ -516,10 +545,20 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
   const int bh = row / nb, r = row % nb, h = bh % Hq;
   const int n = causal ? r + 1 : nb;
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + (size_t)grp * P;
-  const int bar = 1 + grp;
-  auto sync = [bar] {
-    if (RPC == 1) __syncthreads();
-    else asm volatile("bar.sync %0, %1;" ::"r"(bar), "n"(NT) : "memory");
+  // each group syncs on its own named barrier (1 + grp), named by a constant so
+  // that the kernel reserves only the barriers it uses
+  static_assert(RPC == 1 || RPC == 2 || RPC == 4, "one to four rows per CTA");
+  auto sync = [grp] {
+    if (RPC == 1) {
+      __syncthreads();
+      return;
+    }
+    switch (grp) {
+      case 0: asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); break;
+      case 1: asm volatile("bar.sync 2, %0;" ::"n"(NT) : "memory"); break;
+      case 2: asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory"); break;
+      default: asm volatile("bar.sync 4, %0;" ::"n"(NT) : "memory"); break;
+    }
   };
   const SelCut cut = select_row_cut<NT>(scores + (size_t)row * nb, n, r, tau[h], rule, keys,
                                         red[grp], &first_hit[grp], &st[grp], tid, sync);
