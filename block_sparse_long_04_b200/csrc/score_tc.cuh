@@ -10,22 +10,22 @@
 // (XAttention abstract). With `diagonal` set, the query chunk is taken at s*C
 // instead, which sums the tile's main diagonal: the diagonal-pattern variant the
 // DuSA rebuttal (Response to Q2) and the XAttention ablation compare against.
-// The reduction over S*C runs in 64-element chunks
-// through a ring of shared-memory stages; each chunk is four M=128 x N=BN x K=16
-// tcgen05 MMAs into a TMEM accumulator, double-buffered so that the epilogue of
+// The reduction over S*C runs in 64- or 128-element stages
+// through a ring of shared-memory stages; each stage is four or eight
+// K=16 tcgen05 MMAs into a TMEM accumulator, double-buffered so that the epilogue of
 // one column tile overlaps the MMAs of the next.
 //
 // Warp roles (384 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA
 // issuer (warp 1 also owns the TMEM allocation), warps 4-11 = epilogue, two
 // threads per reshaped row (TMEM lane = row): warps 4-7 take the first half of
-// every column tile, warps 8-11 the second, each with its own running row LSE,
+// every column tile, warps 8-11 the second, each with its own reference and sum,
 // merged once at the end; all twelve warps share the finalize.
 //
 // Epilogue (row softmax + block summation, XAttention summary, Approach): for
 // every key block of g = 128/S columns the thread forms the block's base-2
-// log-sum-exp ell[i', c] from its TMEM row, updates the row's running LSE, and
+// log-sum-exp ell[i', c] from its TMEM row, adds the block to its row sum, and
 // writes ell to the workspace. After the sweep all threads of the CTA re-read its
-// ell values (L2-resident) and write
+// ell values and write
 //   scores[r, c] = (1/g) sum_{i' in r} 2^(ell[i', c] - LSE[i']).
 // The (M/S)^2 logits are never stored. Waits are bounded as in attn_tc.cuh.
 //
