@@ -322,13 +322,27 @@ __device__ SelCut select_row_cut(const float* __restrict__ srow, int n, int r, f
   }
   sync();
   bool special = false;
-#pragma unroll 4
-  for (int i = tid; i < n; i += NT) {
-    const float s = srow[i];
+  auto rank_one = [&](int i, float s) {
     const uint32_t rk = desc_rank(s);
     special |= (rk & 0x80000000u) != 0 || !(s <= 3.4028234663852886e38f);   // negative, inf, NaN
     ranks[i] = rk;
+  };
+  // 16-byte loads when the row is 16-byte aligned (the first n & ~3 entries),
+  // so that a thread's loads of the row are few and all in flight together
+  int n4 = 0;
+  if ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
+    n4 = n & ~3;
+    const float4* s4 = reinterpret_cast<const float4*>(srow);
+#pragma unroll 4
+    for (int q = tid; q < n4 / 4; q += NT) {
+      const float4 v = s4[q];
+      rank_one(4 * q, v.x);
+      rank_one(4 * q + 1, v.y);
+      rank_one(4 * q + 2, v.z);
+      rank_one(4 * q + 3, v.w);
+    }
   }
+  for (int i = n4 + tid; i < n; i += NT) rank_one(i, srow[i]);
   if (special) st->special = 1;
   sync();
   if (st->special) {
@@ -526,6 +540,50 @@ __device__ __forceinline__ bool kept_by_cut(float s, int c, int r, const SelCut&
   return c == r || ranks_before(s, c, cut.score, cut.index) || (s == cut.score && c == cut.index);
 }
 
+// Exclusive scan of one int per thread over a group of NT threads (whole warps)
+// that share `sync` as their barrier; red holds NT/32 ints. total = the sum.
+template <int NT, typename Sync>
+__device__ __forceinline__ int group_exclusive_scan_i32(int v, int* red, int tid, Sync sync,
+                                                        int& total) {
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  sync();
+  int before = x - v;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const int t = red[w];
+    if (w < warp) before += t;
+    total += t;
+  }
+  sync();
+  return before;
+}
+
+// Named barrier of group grp (id 1 + grp, NT threads), or the CTA barrier when
+// the CTA holds one group; the ids are constants so that the kernel reserves
+// only the barriers it uses.
+template <int RPC, int NT>
+__device__ __forceinline__ void group_sync(int grp) {
+  static_assert(RPC == 1 || RPC == 2 || RPC == 4, "one to four groups per CTA");
+  if (RPC == 1) {
+    __syncthreads();
+    return;
+  }
+  switch (grp) {
+    case 0: asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); break;
+    case 1: asm volatile("bar.sync 2, %0;" ::"n"(NT) : "memory"); break;
+    case 2: asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory"); break;
+    default: asm volatile("bar.sync 4, %0;" ::"n"(NT) : "memory"); break;
+  }
+}
+
 // One CTA of kSelThreads threads holds RPC rows, a group of NT = kSelThreads /
 // RPC threads per row with its own named barrier; `keys` (dynamic shared
 // memory) holds P 64-bit entries per group. Short rows run four to a CTA (64
@@ -545,21 +603,7 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
   const int bh = row / nb, r = row % nb, h = bh % Hq;
   const int n = causal ? r + 1 : nb;
   uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + (size_t)grp * P;
-  // each group syncs on its own named barrier (1 + grp), named by a constant so
-  // that the kernel reserves only the barriers it uses
-  static_assert(RPC == 1 || RPC == 2 || RPC == 4, "one to four rows per CTA");
-  auto sync = [grp] {
-    if (RPC == 1) {
-      __syncthreads();
-      return;
-    }
-    switch (grp) {
-      case 0: asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); break;
-      case 1: asm volatile("bar.sync 2, %0;" ::"n"(NT) : "memory"); break;
-      case 2: asm volatile("bar.sync 3, %0;" ::"n"(NT) : "memory"); break;
-      default: asm volatile("bar.sync 4, %0;" ::"n"(NT) : "memory"); break;
-    }
-  };
+  auto sync = [grp] { group_sync<RPC, NT>(grp); };   // each group its own barrier
   const SelCut cut = select_row_cut<NT>(scores + (size_t)row * nb, n, r, tau[h], rule, keys,
                                         red[grp], &first_hit[grp], &st[grp], tid, sync);
   if (tid == 0) cuts[row] = cut;
@@ -568,46 +612,79 @@ select_count_kernel(const float* __restrict__ scores, const float* __restrict__ 
 // Rows of at most this many candidates run four to a CTA.
 constexpr int kSelShortRow = 2048;
 
+// One CTA: the rows' counts go through shared memory in chunks of 8192 (loads
+// and stores of consecutive rows by consecutive threads), each thread scanning
+// eight neighbouring counts, the running total carried from chunk to chunk.
 __global__ void __launch_bounds__(1024)
 select_scan_kernel(const SelCut* __restrict__ cuts, int rows, int32_t* __restrict__ row_ptr,
                    int32_t* __restrict__ nnz, long long capacity) {
+  constexpr int kPer = 8, kChunk = kPer * 1024;
+  __shared__ int cnt[kChunk];
   __shared__ int red[32];
-  const int per = (rows + blockDim.x - 1) / blockDim.x;
-  const int lo = threadIdx.x * per, hi = min(rows, lo + per);
-  int seg = 0;
-  for (int i = lo; i < hi; ++i) seg += cuts[i].count;
-  int total;
-  int run = block_exclusive_scan_i32(seg, red, total);
-  const bool over = (long long)total > capacity;
-  for (int i = lo; i < hi; ++i) {
-    row_ptr[i] = over ? 0 : run;
-    run += cuts[i].count;
+  const int tid = threadIdx.x;
+  int carry = 0;
+  for (int base = 0; base < rows; base += kChunk) {
+    const int m = min(kChunk, rows - base);
+    for (int i = tid; i < m; i += 1024) cnt[i] = cuts[base + i].count;
+    __syncthreads();
+    int loc[kPer], seg = 0;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int i = tid * kPer + e;
+      loc[e] = i < m ? cnt[i] : 0;
+      seg += loc[e];
+    }
+    int total;
+    int run = carry + block_exclusive_scan_i32(seg, red, total);
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int i = tid * kPer + e;
+      if (i < m) cnt[i] = run;
+      run += loc[e];
+    }
+    __syncthreads();
+    for (int i = tid; i < m; i += 1024) row_ptr[base + i] = cnt[i];
+    carry += total;
+    __syncthreads();   // cnt is refilled by the next chunk
   }
-  if (threadIdx.x == 0) {
-    row_ptr[rows] = over ? 0 : total;
-    nnz[0] = total;
+  // over capacity: every list is withdrawn (row_ptr all 0) and the error raised;
+  // each entry is zeroed by the thread that wrote it above
+  const bool over = (long long)carry > capacity;
+  if (over)
+    for (int i = tid; i < rows; i += 1024) row_ptr[i] = 0;
+  if (tid == 0) {
+    row_ptr[rows] = over ? 0 : carry;
+    nnz[0] = carry;
     if (over) raise_device_error(2 /* XATTN_ECAPACITY */);
   }
 }
 
+// RPC rows per CTA (a group of NT = kSelThreads / RPC threads per row, each
+// thread a contiguous segment of the row), kept indices in ascending order.
+template <int RPC>
 __global__ void __launch_bounds__(kSelThreads)
 select_fill_kernel(const float* __restrict__ scores, const SelCut* __restrict__ cuts, int nb,
-                   int causal, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx) {
-  __shared__ int red[32];
-  const int row = blockIdx.x;
+                   int causal, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+                   int rows) {
+  constexpr int NT = kSelThreads / RPC;
+  __shared__ int red[RPC][NT / 32];
+  const int grp = (int)threadIdx.x / NT, tid = (int)threadIdx.x % NT;
+  const int row = blockIdx.x * RPC + grp;
+  if (row >= rows) return;   // whole groups leave; the others sync on their own barriers
   const int r = row % nb;
   const int n = causal ? r + 1 : nb;
   const SelCut cut = cuts[row];
   const int base = row_ptr[row];
   if (row_ptr[row + 1] - base != cut.count) return;   // lists withdrawn (capacity)
   const float* srow = scores + (size_t)row * nb;
-  const int per = (n + kSelThreads - 1) / kSelThreads;
-  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  const int per = (n + NT - 1) / NT;
+  const int lo = tid * per, hi = min(n, lo + per);
   auto kept = [&](int c) { return kept_by_cut(srow[c], c, r, cut); };
   int cnt = 0;
   for (int c = lo; c < hi; ++c) cnt += kept(c) ? 1 : 0;
   int total;
-  int pos = block_exclusive_scan_i32(cnt, red, total);
+  int pos = group_exclusive_scan_i32<NT>(cnt, red[grp], tid, [grp] { group_sync<RPC, NT>(grp); },
+                                         total);
   // the row's count bounds the writes even if cuts and scores disagree
   for (int c = lo; c < hi && pos < cut.count; ++c)
     if (kept(c)) col_idx[base + pos++] = c;

@@ -390,6 +390,19 @@ static int launch_select_count(const float* scores, const float* param, int Hq, 
   return cudaGetLastError() == cudaSuccess ? XATTN_OK : XATTN_ECUDA;
 }
 
+// The fill pass: rows of at most 1024 candidates four to a CTA (at most 16 per
+// thread), longer ones one to a CTA.
+static void launch_select_fill(const float* scores, const SelCut* cuts, int nb, int causal,
+                               const int32_t* row_ptr, int32_t* col_idx, long long rows,
+                               cudaStream_t st) {
+  if (nb <= 1024)
+    select_fill_kernel<4><<<(unsigned)((rows + 3) / 4), kSelThreads, 0, st>>>(
+        scores, cuts, nb, causal ? 1 : 0, row_ptr, col_idx, (int)rows);
+  else
+    select_fill_kernel<1><<<(unsigned)rows, kSelThreads, 0, st>>>(
+        scores, cuts, nb, causal ? 1 : 0, row_ptr, col_idx, (int)rows);
+}
+
 // Checks and launches of the per-head selection (count, scan, fill) with the
 // per-row scratch `cuts` supplied by the caller of this helper: the workspace of
 // xattn_select / xattn_select_ex, or the library's fixed array for
@@ -412,8 +425,7 @@ static int select_launch(const float* scores, const float* param, int rule, int 
   const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
   select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
-  select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
-                                                              row_ptr, col_idx);
+  launch_select_fill(scores, cuts, nb, causal, row_ptr, col_idx, rows, st);
   return launch_status();
 }
 
@@ -549,8 +561,7 @@ int xattn_score_select(const void* Q, const void* K, int B, int Hq, int Hkv, int
   const long long cap = col_capacity > (size_t)(1LL << 40) ? (1LL << 40) : (long long)col_capacity;
   select_scan_kernel<<<1, 1024, 0, st>>>(cuts, (int)rows, row_ptr, nnz, cap);
   if (cudaGetLastError() != cudaSuccess) return XATTN_ECUDA;
-  select_fill_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(scores, cuts, nb, causal ? 1 : 0,
-                                                              row_ptr, col_idx);
+  launch_select_fill(scores, cuts, nb, causal, row_ptr, col_idx, rows, st);
   return launch_status();
 }
 
