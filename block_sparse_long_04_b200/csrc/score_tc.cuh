@@ -376,7 +376,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __syncwarp();
   asm volatile("bar.sync 1, 384;" ::: "memory");
   const bool done_ok = !*abort_flag;
-  if (done_ok) {
+  // the plain scoring call leaves this step to score_finalize_kernel (below),
+  // which runs on every SM at once; the fused selection needs the scores here
+  if (SELECT && done_ok) {
     // The (query block r, column c) items of the CTA's rows are spread over the
     // threads: an item's G partials are one aligned run, read by G / VEC
     // neighbouring lanes with one VEC-wide load each, so that a warp's load
@@ -479,6 +481,59 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (PAIR) tmem_dealloc_pair(tmem, L::kTmemCols);
     else tmem_dealloc(tmem, L::kTmemCols);
   }
+}
+
+// The block scores of one (batch, query head, query block r) row from the
+// partials and row LSEs the scoring kernel left in the workspace; the same
+// per-item arithmetic, in the same order, as the scoring kernel's own finalize
+// (G / VEC neighbouring lanes per item, VEC partials each, added by shuffles),
+// so both give the same bits. One CTA of 256 threads per row.
+template <int G>
+__global__ void __launch_bounds__(256)
+score_finalize_kernel(const float* __restrict__ part, const float* __restrict__ lse_ws,
+                      float* __restrict__ scores, int rp, int nb, int causal) {
+  constexpr int VEC = G < 4 ? G : 4;
+  constexpr int TPI = G / VEC;
+  constexpr int IPR = 256 / TPI;
+  constexpr int R = 4;
+  __shared__ float ls[G];
+  const int r = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int sub = tid % TPI, slot = tid / TPI;
+  for (int i = tid; i < G; i += 256) ls[i] = lse_ws[(size_t)bh * rp + (size_t)r * G + i];
+  __syncthreads();
+  const int ncand = causal ? r + 1 : nb;
+  float* srow = scores + ((size_t)bh * nb + r) * nb;
+  const float inv_g = 1.f / (float)G;
+  for (int b0 = 0; b0 < ncand; b0 += R * IPR) {
+    float x[R][VEC];
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int c = b0 + j * IPR + slot;
+      const float* pr = part + part_at<G>(bh, c < ncand ? c : 0, r * G + sub * VEC, rp, nb, causal);
+      if constexpr (VEC == 4) {
+        const float4 t4 = c < ncand ? *reinterpret_cast<const float4*>(pr)
+                                    : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
+        x[j][0] = t4.x; x[j][1] = t4.y; x[j][2] = t4.z; x[j][3] = t4.w;
+      } else {
+        const float2 t2 = c < ncand ? *reinterpret_cast<const float2*>(pr)
+                                    : make_float2(kNegInf, kNegInf);
+        x[j][0] = t2.x; x[j][1] = t2.y;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int c = b0 + j * IPR + slot;
+      const float* lrow = ls + sub * VEC;
+      float a = 0.f;
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) a += c < ncand ? ex2(x[j][u] - lrow[u]) : 0.f;
+#pragma unroll
+      for (int o = TPI / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (sub == 0 && c < ncand) srow[c] = a * inv_g;
+    }
+  }
+  if (causal)
+    for (int c = ncand + tid; c < nb; c += 256) srow[c] = 0.f;
 }
 
 }  // namespace xattn

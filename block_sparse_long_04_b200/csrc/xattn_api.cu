@@ -144,6 +144,9 @@ int launch_score_tc_mode(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, i
     kern<<<dim3(RT, B * Hq), kScoreTcThreads, smem, st>>>(mq, mk, Hq, Hkv, M, causal, diagonal,
                                                          sl2, part, lse_ws, scores, fs.param,
                                                          fs.rule, fs.cuts);
+    if (!SELECT)
+      score_finalize_kernel<G><<<dim3((unsigned)(M / 128), (unsigned)(B * Hq)), 256, 0, st>>>(
+          part, lse_ws, scores, rp, M / 128, causal);
     return launch_status();
   }
   // pairs of heads: grid (2 * RT, B*Hq/2); pairs of row tiles: (2 * ceil(RT/2), B*Hq)
@@ -162,6 +165,11 @@ int launch_score_tc_mode(const bf16* Q, const bf16* K, int B, int Hq, int Hkv, i
   if (cudaLaunchKernelEx(&cfg, kern, mq, mk, Hq, Hkv, M, causal, diagonal, sl2, part, lse_ws,
                          scores, fs.param, fs.rule, fs.cuts) != cudaSuccess)
     return XATTN_ECUDA;
+  if (!SELECT) {
+    // the block scores from the partials, on every SM at once
+    score_finalize_kernel<G><<<dim3((unsigned)(M / 128), (unsigned)(B * Hq)), 256, 0, st>>>(
+        part, lse_ws, scores, rp, M / 128, causal);
+  }
   return launch_status();
 }
 
