@@ -523,10 +523,11 @@ def main():
                  torch.empty(xa.xattn_select_group_workspace_size(w.B, w.Hq, w.Hkv, w.nb),
                              dtype=torch.uint8, device=dev))
 
-    # unfused: score 1, select 3 (count, scan, fill), attention 1;
+    # unfused: score 2 (the sweep, then the block scores from its partials),
+    # select 3 (count, scan, fill), attention 1;
     # fused: score with row cuts 1, scan 1, fill 1, attention 1
-    # grouped: score 1, select 4 (count, group count, scan, group fill), attention 1
-    launches_per_step = 6 if a.group_select else (4 if a.fused_select else 5)
+    # grouped: score 2, select 4 (count, group count, scan, group fill), attention 1
+    launches_per_step = 7 if a.group_select else (4 if a.fused_select else 6)
     clk = ClockSampler(local).__enter__()      # started early: nvidia-smi is slow to start
     try:
         step, evs, t0, t1 = time_layer(xa, L, ss, sa, stream, a.steps, a.warmup,
